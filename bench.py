@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the differential-attention forward on B200.
+
+One step = the whole prefill hot path over one batch of the 3B-like workload
+(B=4, N=4096, H=12 diff heads, d=128, V width 256, causal, bf16): the lambda
+kernel, then the fused dual-map prefill kernel (DiffAttn + RMSNorm + scale).
+The same run also times the decode kernel pair on the KV-cache workload (64
+sequences x 12 heads, lengths ~ U{1024..32768}) and reports its HBM GB/s.
+
+Prints ONE JSON line on rank 0.  `value` is whole-job prefill TFLOP/s with the
+metric's FLOP convention (16*N^2*d per head, half for causal); the roofline
+uses the algorithmic count (12*N^2*d per head, half for causal).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs as one process per GPU under torch.distributed.run; each rank
+processes its own batch (replicas, weak scaling; the path has no exchange
+step), and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DiffAttn fwd TFLOP/s & % BF16 tensor peak (prefill); decode HBM GB/s, 1×B200"
+WORKLOAD = "prefill_3b"
+DECODE_WORKLOAD = "decode_64x12"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_flops(B, N, H, d, causal, convention):
+    per_head = (16.0 if convention == "metric" else 12.0) * N * N * d
+    return per_head * B * H * (0.5 if causal else 1.0)
+
+
+def prefill_row_flops(N, d, causal, convention):
+    return (16.0 if convention == "metric" else 12.0) * N * d * (0.5 if causal else 1.0)
+
+
+def read_profile_traffic(kernel_tag: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current kernel source."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
+    src = os.path.join(ROOT, "differential_attention_04_b200", "csrc",
+                       "prefill_sm100.cu" if kernel_tag.startswith("prefill") else "decode.cu")
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    want = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != want:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s, p in zip(sm, pw)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_rows_sample(inp, n_rows, seed=0):
+    """Run the float64 oracle on n_rows query rows of one head; returns seconds."""
+    import numpy as np
+
+    import oracle.diffattn_ref as ref
+    from differential_attention_04_b200 import workloads as wl
+
+    f = wl.to_f64
+    B, N, H = inp.q.shape[:3]
+    rng = np.random.default_rng(seed)
+    b, h = int(rng.integers(0, B)), int(rng.integers(0, H))
+    rows = np.sort(rng.choice(N, size=min(n_rows, N), replace=False))
+    qh, kh, vh = f(inp.q[b:b + 1, :, h:h + 1]), f(inp.k[b:b + 1, :, h:h + 1]), f(inp.v[b:b + 1, :, h:h + 1])
+    lam = ref.lambda_reparam(f(inp.lq1), f(inp.lk1), f(inp.lq2), f(inp.lk2), inp.lambda_init)
+    t0 = time.perf_counter()
+    ref.diffattn_fwd(qh, kh, vh, lam, inp.lambda_init, f(inp.rms_w), inp.eps, inp.causal, rows=rows)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp, budget_s):
+    """The oracle as it stands on a bounded sample of the workload (query rows of one head)."""
+    N, d = inp.q.shape[1], inp.q.shape[4]
+    rows = 256
+    t = oracle_rows_sample(inp, rows, seed=0)
+    rows_total, secs = rows, t
+    seed = 1
+    while secs < budget_s:
+        n = int(min(N, max(64, rows * (budget_s - secs) / max(t, 1e-3) / 4)))
+        t = oracle_rows_sample(inp, n, seed=seed)
+        rows_total += n
+        secs += t
+        seed += 1
+    flops = rows_total * prefill_row_flops(N, d, inp.causal, "metric")
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows_total} query rows (each against all {N} keys, both maps materialised) of "
+                      f"{seed} seeded (batch, head) pairs of the {WORKLOAD} workload, {secs:.1f} s of CPU work; "
+                      f"FLOPs per row counted with the metric convention 16*N*d/2"}
+
+
+# --------------------------------------------------------------- reference --
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+
+    from differential_attention_04_b200 import workloads as wl
+
+    torch.manual_seed(0)
+    inp = wl.make_prefill_case(args.workload, device="cpu")
+    N, d = inp.q.shape[1], inp.q.shape[4]
+    # size each step so that warm-up + timed steps take about two minutes
+    t_cal = oracle_rows_sample(inp, 64, seed=999)
+    per_row = t_cal / 64
+    total_steps = max(1, args.steps + args.warmup)
+    rows = int(max(8, min(N, 120.0 / total_steps / per_row)))
+    for i in range(args.warmup):
+        oracle_rows_sample(inp, rows, seed=i)
+    secs = 0.0
+    for i in range(args.steps):
+        secs += oracle_rows_sample(inp, rows, seed=1000 + i)
+    flops = args.steps * rows * prefill_row_flops(N, d, inp.causal, "metric")
+    value = flops / secs / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{args.workload}: float64 CPU oracle, {rows} query rows of one head per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{rows} query rows per step (each against all {N} keys) of one seeded "
+                                   f"(batch, head) of {args.workload}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- ours --
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from differential_attention_04_b200 import api
+    from differential_attention_04_b200 import workloads as wl
+    from differential_attention_04_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if rank == 0:
+        build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist.barrier()
+        if rank != 0:
+            build()  # already built by rank 0; just loads
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    inp = wl.make_prefill_case(args.workload, seed=1234 + rank, device=dev)
+    B, N, H, _, d = inp.q.shape
+    lam = torch.empty(1, dtype=torch.float32, device=dev)
+    y = torch.empty_like(inp.v)
+
+    def step():
+        api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init, out=lam)
+        api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for i in range(K):
+        api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init, out=lam)
+        ev[i][0].record()
+        api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
+        ev[i][1].record()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    status = api.device_status()
+    if status != api.OK:
+        raise SystemExit(f"kernel status {status}")
+
+    ms_step = ms_total / K
+    flops_metric = prefill_flops(B, N, H, d, inp.causal, "metric")
+    flops_alg = prefill_flops(B, N, H, d, inp.causal, "algorithmic")
+    value = world * flops_metric / (ms_step * 1e-3) / 1e12
+    achieved = flops_alg / (kern_ms * 1e-3) / 1e12
+    traffic = read_profile_traffic("prefill_sm100_prefill_3b")
+
+    # end to end through the public API: pinned host inputs, H2D inside the timed region, D2H of the output
+    E = max(1, args.e2e_steps)
+    host = {n: getattr(inp, n).cpu().pin_memory() for n in ("q", "k", "v", "lq1", "lk1", "lq2", "lk2", "rms_w")}
+    dbuf = {n: torch.empty_like(getattr(inp, n)) for n in host}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = y_host.numel() * y_host.element_size()
+
+    def e2e_step():
+        for n, t in host.items():
+            dbuf[n].copy_(t, non_blocking=True)
+        api.diffattn_lambda(dbuf["lq1"], dbuf["lk1"], dbuf["lq2"], dbuf["lk2"], inp.lambda_init, out=lam)
+        api.diffattn_fwd(dbuf["q"], dbuf["k"], dbuf["v"], lam, inp.lambda_init, dbuf["rms_w"], inp.eps,
+                         inp.causal, out=y)
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(E):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / E
+    e2e_value = world * flops_metric / (e2e_ms * 1e-3) / 1e12
+    del dbuf, host, y_host
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload}: B={B} N={N} H={H} d={d} V width {2 * d} "
+                        f"{'causal' if inp.causal else 'no mask'} bf16, per rank",
+            "flops_per_step_metric": flops_metric, "flops_per_step_algorithmic": flops_alg,
+            "flop_convention": "value: 16*N^2*d per head (half for causal), as the metric states; "
+                               "roofline: algorithmic 12*N^2*d per head (half for causal)",
+            "l2": f"inputs larger than L2: q+k+v = {3 * inp.q.numel() * 2 / 1e6:.0f} MB per step > 126 MB",
+            "parallelism": f"replicas x{world} (one process per GPU, no collective on the path)",
+        },
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "prefill_sm100_kernel<128>", "kernel_ms": kern_ms,
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+
+    if not args.no_decode:
+        line["decode"] = bench_decode(api, wl, dev, peaks, peak_src, rank, max_over_ranks, barrier, world)
+    del inp, y
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_inp = wl.make_prefill_case(args.workload, seed=1234, device="cpu")
+        line["cpu_baseline"] = cpu_baseline(cpu_inp, args.cpu_budget_s)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_decode(api, wl, dev, peaks, peak_src, rank, max_over_ranks, barrier, world, steps=20):
+    import torch
+
+    inp = wl.make_decode_case(DECODE_WORKLOAD, seed=4321 + rank, device=dev)
+    S, H, _, d = inp.q.shape
+    T = int(inp.seqlens.sum())
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+    ws = torch.empty(api.decode_workspace_size(S, H, d, inp.max_seqlen), dtype=torch.uint8, device=dev)
+    y = torch.empty((S, H, 2 * d), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        api.diffattn_decode(inp.q, inp.k_cache, inp.v_cache, inp.cu_seqlens, inp.max_seqlen, lam, inp.lambda_init,
+                            inp.rms_w, inp.eps, workspace=ws, out=y)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b)) / steps
+    kv_bytes = T * H * (2 * d + 2 * d) * 2
+    io_bytes = S * H * 2 * d * 2 * 2
+    alg = kv_bytes + io_bytes
+    gbs = alg / (ms * 1e-3) / 1e9
+    traffic = read_profile_traffic("decode_decode_64x12")
+    return {
+        "metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+        "workload": f"{DECODE_WORKLOAD}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
+                    f"({kv_bytes / 1e9:.2f} GB per step)",
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": "decode_partial_kernel + decode_combine_kernel",
+                     "algorithmic_bytes": alg, "peak_source": f"{peak_src} HBM copy"},
+        "gpu_launches": 2 * steps,
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

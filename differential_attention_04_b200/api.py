@@ -1,0 +1,118 @@
+"""Python binding of the C ABI in include/diffattn.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Tensors are passed by device pointer on the current torch stream;
+the functions return immediately (stream-ordered), like the C calls.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import lib
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
+F32, BF16 = 0, 1
+
+
+class DiffAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = lib().diffattn_status_string(status).decode()
+        super().__init__(f"{fn} failed: {msg} (status {status})")
+        self.status = status
+
+
+def _check(fn: str, status: int) -> None:
+    if status != OK:
+        raise DiffAttnError(fn, status)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dev(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def diffattn_lambda(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor, lk2: torch.Tensor,
+                    lambda_init: float, out: torch.Tensor | None = None) -> torch.Tensor:
+    """lambda = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init, as a device fp32 scalar (shape [1])."""
+    _dev(lq1, lk1, lq2, lk2)
+    for t in (lq1, lk1, lq2, lk2):
+        if t.dtype != torch.float32:
+            raise ValueError("lambda vectors must be float32")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=lq1.device)
+    _check("diffattn_lambda", lib().diffattn_lambda(
+        _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), lq1.numel(), float(lambda_init), _ptr(out), _stream()))
+    return out
+
+
+def diffattn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor, lambda_init: float,
+                 rms_w: torch.Tensor, eps: float = 1e-5, causal: bool = True,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """Prefill.  q, k: [B, N, H, 2, d]; v: [B, N, H, 2d]; lam: device fp32 scalar; rms_w: fp32 [2d]."""
+    _dev(q, k, v, lam, rms_w)
+    B, N, H, two, d = q.shape
+    if two != 2 or k.shape != q.shape or tuple(v.shape) != (B, N, H, 2 * d):
+        raise ValueError("shapes must be q, k: [B, N, H, 2, d] and v: [B, N, H, 2d]")
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype == torch.float32:
+        dt = F32
+    else:
+        raise ValueError("dtype must be bfloat16 or float32")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype")
+    if out is None:
+        out = torch.empty_like(v)
+    _check("diffattn_fwd", lib().diffattn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)), _ptr(lam),
+        float(lambda_init), _ptr(rms_w), float(eps), _stream()))
+    return out
+
+
+def decode_workspace_size(S: int, H: int, d: int, max_seqlen: int) -> int:
+    return int(lib().diffattn_decode_workspace_size(S, H, d, max_seqlen))
+
+
+def diffattn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, cu_seqlens: torch.Tensor,
+                    max_seqlen: int, lam: torch.Tensor, lambda_init: float, rms_w: torch.Tensor,
+                    eps: float = 1e-5, workspace: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode.  q: [S, H, 2, d]; k_cache: [T, H, 2, d]; v_cache: [T, H, 2d]; cu_seqlens: int32 [S + 1]."""
+    _dev(q, k_cache, v_cache, cu_seqlens, lam, rms_w)
+    S, H, two, d = q.shape
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.numel() != S + 1:
+        raise ValueError("cu_seqlens must be int32 with S + 1 entries")
+    need = decode_workspace_size(S, H, d, max_seqlen)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((S, H, 2 * d), dtype=q.dtype, device=q.device)
+    _check("diffattn_decode", lib().diffattn_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
+        _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _ptr(workspace), workspace.numel(),
+        _stream()))
+    return out
+
+
+def device_status() -> int:
+    """Synchronise the device and return (and clear) the kernels' status word."""
+    v = ctypes.c_int(0)
+    _check("diffattn_device_status", lib().diffattn_device_status(ctypes.byref(v)))
+    return v.value
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    _check("diffattn_set_wait_limit_ns", lib().diffattn_set_wait_limit_ns(int(limit_ns)))

@@ -1,0 +1,172 @@
+// C-ABI entry points declared in include/diffattn.h: argument validation,
+// TMA descriptor encoding, the device status word, and dispatch to the
+// kernels.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "diffattn.h"
+#include "internal.h"
+
+namespace diffattn {
+namespace {
+
+// Device-side status word: kernels record DIFFATTN_ERR_TIMEOUT here.
+__device__ int g_status_word = 0;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? DIFFATTN_OK : DIFFATTN_ERR_CUDA; }
+
+// Address of this device's status word (looked up once per device).
+cudaError_t status_ptr(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return e;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return cudaSuccess;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 map over a row-major tensor with dims (innermost first) d0..d3,
+// box = 64 x 1 x 128 x 1 elements, 128-byte swizzle, zero fill out of bounds.
+bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool fits_i32(long long x) { return x >= 0 && x < (1ll << 31); }
+
+}  // namespace
+}  // namespace diffattn
+
+using namespace diffattn;
+
+extern "C" {
+
+int diffattn_version(void) { return 100; }
+
+const char* diffattn_status_string(int s) {
+  switch (s) {
+    case DIFFATTN_OK: return "ok";
+    case DIFFATTN_ERR_INVALID_ARG: return "invalid argument";
+    case DIFFATTN_ERR_UNSUPPORTED: return "unsupported dtype or size";
+    case DIFFATTN_ERR_CUDA: return "CUDA error";
+    case DIFFATTN_ERR_TIMEOUT: return "a kernel wait timed out";
+    case DIFFATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int diffattn_set_wait_limit_ns(long long limit_ns) {
+  if (limit_ns < 0) return DIFFATTN_ERR_INVALID_ARG;
+  g_wait_limit_ns.store(limit_ns == 0 ? 2000000000ull : static_cast<unsigned long long>(limit_ns));
+  return DIFFATTN_OK;
+}
+
+int diffattn_device_status(int* status_out) {
+  if (!status_out) return DIFFATTN_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  *status_out = v;
+  return DIFFATTN_OK;
+}
+
+int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
+                    float lambda_init, float* lambda_out, cudaStream_t stream) {
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !lambda_out) return DIFFATTN_ERR_INVALID_ARG;
+  if (d < 1 || d > 4096) return DIFFATTN_ERR_INVALID_ARG;
+  return cuda_status(launch_lambda(lq1, lk1, lq2, lk2, d, lambda_init, lambda_out, stream));
+}
+
+int diffattn_fwd(const void* q, const void* k, const void* v, void* o, int dtype, int B, int N, int H, int d,
+                 int causal, const float* lambda, float lambda_init, const float* rms_w, float eps,
+                 cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 0 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (dtype != DIFFATTN_F32 && dtype != DIFFATTN_BF16) return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (N == 0) return DIFFATTN_OK;
+  if (!q || !k || !v || !o || !lambda || !rms_w) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DIFFATTN_ERR_INVALID_ARG;
+  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (dtype == DIFFATTN_F32) {
+    if (d > 128) return DIFFATTN_ERR_UNSUPPORTED;
+    return cuda_status(launch_prefill_simt_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                               static_cast<const float*>(v), static_cast<float*>(o), B, N, H, d,
+                                               causal, lambda, lambda_init, rms_w, eps, stream));
+  }
+  if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
+      !encode_4d(&tv, v, 2ull * d, H, N, B))
+    return DIFFATTN_ERR_CUDA;
+  DevCtl ctl;
+  cudaError_t e = status_ptr(&ctl.status);
+  if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  ctl.limit_ns = g_wait_limit_ns.load();
+  return cuda_status(
+      launch_prefill_sm100(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, ctl, stream));
+}
+
+size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen) {
+  return decode_workspace_bytes(S, H, d, max_seqlen);
+}
+
+int diffattn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens, int max_seqlen,
+                    void* o, int S, int H, int d, const float* lambda, float lambda_init, const float* rms_w,
+                    float eps, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (S < 1 || H < 1 || d < 1 || max_seqlen < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !cu_seqlens || !o || !lambda || !rms_w) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (S > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  const size_t need = decode_workspace_bytes(S, H, d, max_seqlen);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
+  return cuda_status(launch_decode(q, k_cache, v_cache, cu_seqlens, max_seqlen, o, S, H, d, lambda, lambda_init,
+                                   rms_w, eps, workspace, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,279 @@
+// Split-KV decode (query length 1) over a packed bf16 KV cache, d = 128.
+//
+// Per (sequence, head) it computes the DiffAttn equation for one query (page
+// "Differential Transformer: Canceling Context Noise with Differential
+// Attention", "Cancelling Context Noise Through Attention Map Subtraction";
+// peer review "Differential Transformer", Summary, Eq. 1) against every cached
+// key of the sequence, then the headwise RMSNorm and the (1 - lambda_init)
+// scale (Eq. 3).
+//
+// The work is bandwidth-bound (1 KiB of K and V per key and head, about 1.5
+// flop per byte), so it runs on CUDA cores:
+//   * decode_partial_kernel: one CTA per (key chunk, head, sequence).  Each
+//     warp streams its keys with 16-byte non-allocating loads, 8 keys in
+//     flight per lane group; lane l holds elements [8l, 8l+8) of the 256-wide
+//     K row (lanes 0-15: map 1, lanes 16-31: map 2) and of the V row.  The 8
+//     partial dot products are reduced across 16 lanes with a transposing
+//     shuffle tree (8 shuffles for 8 keys), and each map keeps its own online
+//     softmax state in the log2 domain.  The 4 warps merge, and the CTA writes
+//     (m1, l1, m2, l2, o1[256], o2[256]) for its chunk to the workspace.
+//   * decode_combine_kernel: one CTA per (head, sequence) merges the chunks
+//     with the log-sum-exp rescale per map, forms o1/l1 - lambda o2/l2, and
+//     applies the RMSNorm and scale.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace diffattn {
+
+namespace {
+constexpr int kD = 128;                 // per-map width
+constexpr int kDV = 2 * kD;             // value / output width
+constexpr int kWarps = 4;
+constexpr int kGroup = 8;               // keys in flight per warp
+constexpr int kKeysPerWarp = 128;
+constexpr int kChunk = kWarps * kKeysPerWarp;  // keys per CTA
+constexpr int kRecFloats = 4 + 2 * kDV;        // m1, l1, m2, l2, o1[256], o2[256]
+constexpr float kLog2e = 1.4426950408889634f;
+}  // namespace
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  f[0] = bf16lo_to_f32(u.x); f[1] = bf16hi_to_f32(u.x);
+  f[2] = bf16lo_to_f32(u.y); f[3] = bf16hi_to_f32(u.y);
+  f[4] = bf16lo_to_f32(u.z); f[5] = bf16hi_to_f32(u.z);
+  f[6] = bf16lo_to_f32(u.w); f[7] = bf16hi_to_f32(u.w);
+}
+
+__global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
+    const int* __restrict__ cu_seqlens, int max_seqlen, int H, int max_chunks, float* __restrict__ ws) {
+  const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int lo = cu_seqlens[s];
+  const int L = min(cu_seqlens[s + 1] - lo, max_seqlen);
+  const int c0 = chunk * kChunk;
+  if (c0 >= L && !(chunk == 0)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4;  // 0: map 1, 1: map 2
+  const int hl = lane & 15;
+
+  // This lane's slice of q (map `half`, elements [8*hl, 8*hl + 8)), pre-scaled
+  // so that scores come out in log2 units: s * log2(e) / sqrt(d).
+  float qf[8];
+  {
+    const uint4 qu = *reinterpret_cast<const uint4*>(q + (static_cast<size_t>(s) * H + h) * kDV + 8 * lane);
+    bf16x8_to_f32(qu, qf);
+    const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qf[i] *= sc;
+  }
+
+  float m1 = -INFINITY, m2 = -INFINITY;  // running max per map (same in all lanes)
+  float lsum = 0.f;                      // this lane's share of its map's running sum
+  float o1[8], o2[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o1[i] = o2[i] = 0.f;
+
+  const size_t row_stride = static_cast<size_t>(H) * kDV;  // elements between consecutive keys
+  const int kbeg = c0 + warp * kKeysPerWarp;
+  const int kend = min(L, kbeg + kKeysPerWarp);
+  const __nv_bfloat16* kbase = kc + static_cast<size_t>(lo) * row_stride + static_cast<size_t>(h) * kDV + 8 * lane;
+  const __nv_bfloat16* vbase = vc + static_cast<size_t>(lo) * row_stride + static_cast<size_t>(h) * kDV + 8 * lane;
+
+  for (int k0 = kbeg; k0 < kend; k0 += kGroup) {
+    uint4 kr[kGroup], vr[kGroup];
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      const int key = k0 + g;
+      if (key < kend) {
+        kr[g] = ldg_stream_v4(kbase + static_cast<size_t>(key) * row_stride);
+        vr[g] = ldg_stream_v4(vbase + static_cast<size_t>(key) * row_stride);
+      } else {
+        kr[g] = make_uint4(0, 0, 0, 0);
+        vr[g] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    // partial dot products of this lane's 8 elements, one per key
+    float part[kGroup];
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      float kf[8];
+      bf16x8_to_f32(kr[g], kf);
+      float a = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a = fmaf(qf[i], kf[i], a);
+      part[g] = a;
+    }
+    // Transposing reduction over the 16 lanes of each half-warp: after the
+    // xor-8, xor-4 and xor-2 steps lane hl holds key g = 4*b3 + 2*b2 + b1
+    // (bits of hl) summed over 8 lanes; the xor-1 step completes the sum.
+    const bool b3 = (hl >> 3) & 1, b2 = (hl >> 2) & 1, b1 = (hl >> 1) & 1;
+    float r4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float keep = b3 ? part[4 + i] : part[i];
+      const float give = b3 ? part[i] : part[4 + i];
+      r4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+    }
+    float r2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float keep = b2 ? r4[2 + i] : r4[i];
+      const float give = b2 ? r4[i] : r4[2 + i];
+      r2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+    }
+    float sc;
+    {
+      const float keep = b1 ? r2[1] : r2[0];
+      const float give = b1 ? r2[0] : r2[1];
+      sc = keep + __shfl_xor_sync(0xffffffffu, give, 2);
+    }
+    sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+    const int my_key = 4 * b3 + 2 * b2 + b1;  // lanes 2g and 2g+1 of each half hold key g
+    if (k0 + my_key >= kend) sc = -INFINITY;
+
+    // group max per map, shared with the other half
+    float mx = sc;
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mx_other = __shfl_xor_sync(0xffffffffu, mx, 16);
+    const float gm1 = half ? mx_other : mx;
+    const float gm2 = half ? mx : mx_other;
+    const float mn1 = fmaxf(m1, gm1), mn2 = fmaxf(m2, gm2);
+    const float al1 = fast_exp2(m1 - mn1), al2 = fast_exp2(m2 - mn2);  // exp2(-inf) = 0
+    m1 = mn1;
+    m2 = mn2;
+    const float p = fast_exp2(sc - (half ? mn2 : mn1));  // 0 for masked keys
+    lsum = lsum * (half ? al2 : al1) + ((lane & 1) ? 0.f : p);
+
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      o1[i] *= al1;
+      o2[i] *= al2;
+    }
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      const float p1 = __shfl_sync(0xffffffffu, p, 2 * g);
+      const float p2 = __shfl_sync(0xffffffffu, p, 16 + 2 * g);
+      float vf[8];
+      bf16x8_to_f32(vr[g], vf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o1[i] = fmaf(p1, vf[i], o1[i]);
+        o2[i] = fmaf(p2, vf[i], o2[i]);
+      }
+    }
+  }
+
+  // running sums per map: sum the lanes of each half
+  float l = lsum;
+  l += __shfl_xor_sync(0xffffffffu, l, 8);
+  l += __shfl_xor_sync(0xffffffffu, l, 4);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  const float l_other = __shfl_xor_sync(0xffffffffu, l, 16);
+  const float l1 = half ? l_other : l, l2 = half ? l : l_other;
+
+  // merge the warps of the CTA
+  __shared__ float sm_m[kWarps][2], sm_l[kWarps][2];
+  __shared__ float sm_o[kWarps][2][kDV];
+  if (lane == 0) {
+    sm_m[warp][0] = m1; sm_m[warp][1] = m2;
+    sm_l[warp][0] = l1; sm_l[warp][1] = l2;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sm_o[warp][0][8 * lane + i] = o1[i];
+    sm_o[warp][1][8 * lane + i] = o2[i];
+  }
+  __syncthreads();
+  float* rec = ws + ((static_cast<size_t>(s) * H + h) * max_chunks + chunk) * kRecFloats;
+  for (int mp = 0; mp < 2; ++mp) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][mp]);
+    float f[kWarps];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) f[w] = (M == -INFINITY) ? 0.f : fast_exp2(sm_m[w][mp] - M);
+    for (int c = threadIdx.x; c < kDV; c += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) acc = fmaf(f[w], sm_o[w][mp][c], acc);
+      rec[4 + mp * kDV + c] = acc;
+    }
+    if (threadIdx.x == 0) {
+      float Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) Ls = fmaf(f[w], sm_l[w][mp], Ls);
+      rec[2 * mp] = M;
+      rec[2 * mp + 1] = Ls;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __restrict__ ws,
+                                                             const int* __restrict__ cu_seqlens, int max_seqlen,
+                                                             int H, int max_chunks, __nv_bfloat16* __restrict__ o,
+                                                             const float* __restrict__ lambda_ptr, float lambda_init,
+                                                             const float* __restrict__ rms_w, float eps) {
+  const int h = blockIdx.x, s = blockIdx.y;
+  const int c = threadIdx.x;
+  const int L = min(cu_seqlens[s + 1] - cu_seqlens[s], max_seqlen);
+  const int nch = max(1, (L + kChunk - 1) / kChunk);
+  const float* rec0 = ws + (static_cast<size_t>(s) * H + h) * max_chunks * kRecFloats;
+  float M1 = -INFINITY, M2 = -INFINITY;
+  for (int i = 0; i < nch; ++i) {
+    M1 = fmaxf(M1, rec0[i * kRecFloats + 0]);
+    M2 = fmaxf(M2, rec0[i * kRecFloats + 2]);
+  }
+  float L1 = 0.f, L2 = 0.f, O1 = 0.f, O2 = 0.f;
+  for (int i = 0; i < nch; ++i) {
+    const float* r = rec0 + i * kRecFloats;
+    const float f1 = fast_exp2(r[0] - M1), f2 = fast_exp2(r[2] - M2);
+    L1 = fmaf(f1, r[1], L1);
+    L2 = fmaf(f2, r[3], L2);
+    O1 = fmaf(f1, r[4 + c], O1);
+    O2 = fmaf(f2, r[4 + kDV + c], O2);
+  }
+  const float lam = *lambda_ptr;
+  const float ov = O1 / L1 - lam * (O2 / L2);
+  // sum of squares over the 256 channels
+  __shared__ float red[kDV / 32];
+  float ss = ov * ov;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((c & 31) == 0) red[c >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < kDV / 32; ++i) tot += red[i];
+  const float rs = rsqrtf(tot / static_cast<float>(kDV) + eps);
+  o[(static_cast<size_t>(s) * H + h) * kDV + c] = __float2bfloat16_rn((1.0f - lambda_init) * rms_w[c] * ov * rs);
+}
+
+size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen) {
+  if (S <= 0 || H <= 0 || d != kD || max_seqlen <= 0) return 0;
+  const size_t chunks = (static_cast<size_t>(max_seqlen) + kChunk - 1) / kChunk;
+  return static_cast<size_t>(S) * H * chunks * kRecFloats * sizeof(float);
+}
+
+cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
+                          int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
+                          const float* rms_w, float eps, void* workspace, cudaStream_t stream) {
+  (void)d;
+  const int max_chunks = (max_seqlen + kChunk - 1) / kChunk;
+  dim3 grid(max_chunks, H, S);
+  decode_partial_kernel<<<grid, kWarps * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
+      static_cast<const __nv_bfloat16*>(v_cache), cu_seqlens, max_seqlen, H, max_chunks,
+      static_cast<float*>(workspace));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<<<dim3(H, S), kDV, 0, stream>>>(static_cast<const float*>(workspace), cu_seqlens,
+                                                        max_seqlen, H, max_chunks, static_cast<__nv_bfloat16*>(o),
+                                                        lambda, lambda_init, rms_w, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace diffattn

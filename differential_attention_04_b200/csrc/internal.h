@@ -1,0 +1,37 @@
+// Launchers shared between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace diffattn {
+
+// Where kernels record a failed bounded wait, and how long a wait may spin.
+struct DevCtl {
+  int* status;
+  unsigned long long limit_ns;
+};
+
+cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
+                          float lambda_init, float* out, cudaStream_t stream);
+
+// CUDA-core prefill for float32 tensors, any 1 <= d <= 128.
+cudaError_t launch_prefill_simt_f32(const float* q, const float* k, const float* v, float* o, int B, int N, int H,
+                                    int d, int causal, const float* lambda, float lambda_init, const float* rms_w,
+                                    float eps, cudaStream_t stream);
+
+// Tensor-core (tcgen05) prefill for bf16 tensors, d in {64, 128}.  tq/tk map
+// [B, N, H*2, d]; tv maps [B, N, H, 2d]; boxes are 64 columns x 128 rows with
+// 128-byte swizzle.
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                                 int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
+                                 const float* rms_w, float eps, DevCtl ctl, cudaStream_t stream);
+
+// Split-KV decode (bf16, d = 128).
+size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);
+cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
+                          int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
+                          const float* rms_w, float eps, void* workspace, cudaStream_t stream);
+
+}  // namespace diffattn

@@ -1,0 +1,468 @@
+// Fused dual-map differential-attention prefill for sm_100a (bf16 in, fp32
+// accumulate, bf16 out), d in {64, 128}.
+//
+// Computes, per head, the DiffAttn equation (page "Differential Transformer:
+// Canceling Context Noise with Differential Attention", "Cancelling Context
+// Noise Through Attention Map Subtraction"; peer review "Differential
+// Transformer", Summary, Eq. 1), then the headwise RMSNorm over the 2d value
+// channels and the fixed (1 - lambda_init) scale (Eq. 3).  No N x N map is
+// ever written to memory.
+//
+// Work decomposition
+//   A cluster of two CTAs owns one 128-row query tile of one (batch, head).
+//   CTA rank i computes map i+1 only: S_i = Q_i K_i^T on the tensor cores,
+//   its own online softmax (running max m_i and sum l_i per row), and
+//   O_i += P_i V.  Both CTAs stream the same V tiles.  Tensor memory per CTA
+//   (512 columns): S double-buffered in columns [0,128) and [128,256), O_i in
+//   [256, 256 + 2d).  P (bf16) overwrites the upper 64 columns of its S
+//   buffer and feeds the PV product straight from tensor memory.
+//   The epilogue exchanges half of the columns through distributed shared
+//   memory: rank 0 keeps output columns [0, d), rank 1 keeps [d, 2d); each
+//   sends the other half of its O_i/l_i (scaled by -lambda on rank 1), the
+//   two halves of the row's sum of squares are swapped, and each CTA writes
+//   its columns of (1 - lambda_init) * w * O / rms.
+//
+// Warp roles (256 threads)
+//   warp 0: TMA producer for Q_i and K_i      warp 2: TMA producer for V
+//   warp 1: tensor-memory allocator + the single MMA-issuing thread
+//   warp 3: idle                              warps 4-7: softmax + epilogue,
+//                                             one query row per thread
+//
+// Pipeline per key tile j (buffer b = j % 2):
+//   MMA:     S_j (keys 0-63 and 64-127 as two N=64 halves once the ring is
+//            warm) -> commit s_full[b]; wait p_full[b]; O += P_j V_j ->
+//            commit o_ready, v_empty.  The second half of S_{j+2} is issued
+//            only after PV_j has completed, because it overwrites P_j.
+//   softmax: wait s_full[b]; read the 128 scores of its row; mask; lazy
+//            rescale (O is rescaled only when the running max grows by more
+//            than 2^8, after PV_{j-1} has completed); P = exp2(s*c - m);
+//            store P as bf16 into tensor memory; arrive p_full[b].
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace diffattn {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBM = 128;  // query rows per CTA
+constexpr int kBN = 128;  // keys per tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int DV = 2 * D;
+  static constexpr int HALF = D;                 // output columns owned by each CTA
+  static constexpr int QBLK = D / 64;            // 64-column swizzle blocks per Q/K row
+  static constexpr int VBLK = DV / 64;           // 64-column blocks per V row
+  static constexpr int BLK_BYTES = 128 * 128;    // one [128 rows][64 bf16] block
+  static constexpr int Q_BYTES = kBM * D * 2;
+  static constexpr int K_BYTES = kBN * D * 2;
+  static constexpr int V_BYTES = kBN * DV * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + 2 * K_BYTES;
+  static constexpr int OFF_BAR = OFF_V + 2 * V_BYTES;
+  static constexpr int OFF_SSX = OFF_BAR + 256;  // float[128]: partner's sum of squares
+  static constexpr int SMEM_USED = OFF_SSX + 512;
+  static constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
+  static constexpr uint32_t TM_S = 0;            // S buffer b at column 128 * b
+  static constexpr uint32_t TM_O = 256;
+  static constexpr uint32_t TM_COLS = 512;
+  static_assert(kBM * HALF * 4 <= V_BYTES, "exchange buffer must fit in one V stage");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_ready;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+}  // namespace
+
+struct PrefillParams {
+  __nv_bfloat16* o;
+  int N, H, causal, n_qtiles;
+  const float* lambda;
+  float lambda_init;
+  const float* rms_w;
+  float eps;
+  int* status;
+  unsigned long long limit_ns;
+};
+
+// Wait for every tcgen05.ld issued so far and pin 128 registers behind the wait.
+__device__ __forceinline__ void tmem_ld_wait4(uint32_t (&a)[32], uint32_t (&b)[32], uint32_t (&c)[32],
+                                              uint32_t (&d)[32]) {
+  tmem_ld_wait(a);
+  tmem_ld_wait(b);  // no outstanding loads remain: these only order the registers
+  tmem_ld_wait(c);
+  tmem_ld_wait(d);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                         const __grid_constant__ CUtensorMap tv, const PrefillParams p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  float* ssx = reinterpret_cast<float*>(smem + C::OFF_SSX);
+  float* sX = reinterpret_cast<float*>(sV);  // epilogue exchange buffer (V stage 0)
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: map 1, 1: map 2
+  const int qtile = p.n_qtiles - 1 - static_cast<int>(blockIdx.x >> 1);  // heaviest tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int N = p.N;
+  const int n_kvtiles = (N + kBN - 1) / kBN;
+  const int n_kv = p.causal ? min(qtile + 1, n_kvtiles) : n_kvtiles;
+
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+    }
+    mbar_init(&bars->o_ready, 1);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  const WaitCtl wc{p.status, &bars->abort, p.limit_ns};
+  // Drains (after a normal run these return at once) ignore the abort flag.
+  int drain_abort = 0;
+  const WaitCtl wdrain{p.status, &drain_abort, 1000000000ull};
+
+  if (warp == 0) {
+    // ---------------------------------------------------- Q / K producer --
+    if (lane == 0) {
+      const int c1 = 2 * h + static_cast<int>(rank);
+      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+#pragma unroll
+      for (int blk = 0; blk < C::QBLK; ++blk)
+        tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * 64, c1, qtile * kBM, b);
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&bars->k_empty[st], ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
+#pragma unroll
+        for (int blk = 0; blk < C::QBLK; ++blk)
+          tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * 64, c1, j * kBN, b);
+        issued = j + 1;
+      }
+      // make sure nothing is still landing in shared memory before the epilogue reuses it
+      mbar_wait(&bars->q_full, 0, wdrain);
+      for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, wdrain);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // -------------------------------------------------------- V producer --
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&bars->v_empty[st], ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
+#pragma unroll
+        for (int blk = 0; blk < C::VBLK; ++blk)
+          tma_load_4d(sV + st * C::V_BYTES + blk * C::BLK_BYTES, &tv, &bars->v_full[st], blk * 64, h, j * kBN, b);
+        issued = j + 1;
+      }
+      for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, wdrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc_s128 = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_s64 = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      // S_buf[n_lo, n_lo + n_cnt) = Q K[n_lo : n_lo + n_cnt]^T for the K tile in stage `st`
+      auto issue_s = [&](int st, int buf, int n_lo, bool full) {
+        const uint32_t d_tmem = tmem + C::TM_S + 128 * buf + n_lo;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int blk = kk >> 2;
+          const uint32_t koff = (kk & 3) * 32;
+          const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + n_lo * 128 + koff, 16, 1024);
+          umma_ss(d_tmem, ad, bd, full ? idesc_s128 : idesc_s64, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, wc);
+      for (int t = 0; ok && t < min(2, n_kv); ++t) {
+        if (!(ok = mbar_wait(&bars->k_full[t], 0, wc))) break;
+        tc_fence_after();
+        issue_s(t, t, 0, true);
+        umma_commit(&bars->k_empty[t]);
+        umma_commit(&bars->s_full[t]);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int bb = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!(ok = mbar_wait(&bars->v_full[bb], ph, wc))) break;
+        if (!(ok = mbar_wait(&bars->p_full[bb], ph, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t a_tmem = tmem + C::TM_S + 128 * bb + 64 + 8 * kk;
+          const uint64_t bd = smem_desc_sw128(sVa + bb * C::V_BYTES + kk * 2048, C::BLK_BYTES, 1024);
+          umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->v_empty[bb]);
+        umma_commit(&bars->o_ready);
+        if (j + 2 < n_kv) {
+          if (!(ok = mbar_wait(&bars->k_full[bb], ((j + 2) >> 1) & 1, wc))) break;
+          tc_fence_after();
+          issue_s(bb, bb, 0, false);  // keys 0-63: columns already consumed by the softmax
+          if (!(ok = mbar_wait(&bars->o_ready, j & 1, wc))) break;  // PV_j done: P_j is free
+          tc_fence_after();
+          issue_s(bb, bb, 64, false);  // keys 64-127 overwrite P_j
+          umma_commit(&bars->k_empty[bb]);
+          umma_commit(&bars->s_full[bb]);
+        }
+      }
+      // drain: every issued MMA has completed before tensor memory is read or freed
+      umma_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0, wdrain);
+    }
+    __syncwarp();
+  }
+
+  // ------------------------------------------------------------ softmax --
+  const bool is_sm = warp >= 4;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;  // query row within the tile (= TMEM lane)
+  const int qrow = qtile * kBM + r;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  float m_run = -INFINITY, l_run = 0.f;
+  bool sm_ok = true;
+  if (is_sm) {
+    const float sc = kLog2e * rsqrtf(static_cast<float>(D));
+    for (int j = 0; j < n_kv; ++j) {
+      const int bb = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      if (!(sm_ok = mbar_wait(&bars->s_full[bb], ph, wc))) break;
+      tc_fence_after();
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      const uint32_t sb = tl + C::TM_S + 128 * bb;
+      tmem_ld32(sb + 0, s0);
+      tmem_ld32(sb + 32, s1);
+      tmem_ld32(sb + 64, s2);
+      tmem_ld32(sb + 96, s3);
+      tmem_ld_wait4(s0, s1, s2, s3);
+      float x[128];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        x[i] = __uint_as_float(s0[i]);
+        x[32 + i] = __uint_as_float(s1[i]);
+        x[64 + i] = __uint_as_float(s2[i]);
+        x[96 + i] = __uint_as_float(s3[i]);
+      }
+      const int key0 = j * kBN;
+      if (key0 + kBN > N || (p.causal && j == qtile)) {
+        const int lim = p.causal ? min(N - 1, qrow) : N - 1;  // last visible key
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (key0 + i > lim) x[i] = -INFINITY;
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, x[i]);
+      const float t_mx = mx * sc;
+      if (j == 0) {
+        m_run = t_mx;
+      } else {
+        const bool need = t_mx > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? fast_exp2(m_run - t_mx) : 1.0f;
+          if (!(sm_ok = mbar_wait(&bars->o_ready, (j - 1) & 1, wc))) break;  // PV_{j-1} done
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < C::DV / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tl + C::TM_O + 32 * c, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tl + C::TM_O + 32 * c, ov);
+          }
+          tmem_st_wait();
+          l_run *= alpha;
+          if (need) m_run = t_mx;
+        }
+      }
+      const float mneg = -m_run;
+      uint32_t pk[32];
+      float lsum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = fast_exp2(fmaf(x[64 * half + 2 * i], sc, mneg));
+          const float p1 = fast_exp2(fmaf(x[64 * half + 2 * i + 1], sc, mneg));
+          lsum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(sb + 64 + 32 * half, pk);
+      }
+      tmem_st_wait();
+      l_run += lsum;
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[bb]);
+    }
+    if (sm_ok) sm_ok = mbar_wait(&bars->o_ready, (n_kv - 1) & 1, wc);  // last PV done
+    tc_fence_after();
+  }
+
+  // ----------------------------------------------------------- epilogue --
+  cluster_sync_all();  // both CTAs: main loops drained, V stage 0 free for the exchange
+  const float lam = *p.lambda;
+  const float inv = (rank == 0) ? 1.0f / l_run : -lam / l_run;
+  const int own0 = (rank == 0) ? 0 : C::HALF;   // columns this CTA finishes
+  const int send0 = (rank == 0) ? C::HALF : 0;  // columns the partner finishes
+  constexpr int NCH = C::HALF / 4;              // float4 chunks per exchange row
+  if (is_sm) {
+    const uint32_t remote = map_to_cta(smem_u32(sX), rank ^ 1u);
+#pragma unroll
+    for (int c = 0; c < C::HALF / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld32(tl + C::TM_O + send0 + 32 * c, ov);
+      tmem_ld_wait(ov);
+#pragma unroll
+      for (int f = 0; f < 8; ++f) {
+        const int chunk = (c * 8 + f) ^ (r % NCH);
+        st_cluster_v4(remote + static_cast<uint32_t>((r * C::HALF + chunk * 4) * 4),
+                      __uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                      __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
+      }
+    }
+  }
+  cluster_sync_all();  // exchanged halves visible
+  float y[C::HALF];
+  float ss = 0.f;
+  if (is_sm) {
+#pragma unroll
+    for (int c = 0; c < C::HALF / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld32(tl + C::TM_O + own0 + 32 * c, ov);
+      tmem_ld_wait(ov);
+#pragma unroll
+      for (int f = 0; f < 8; ++f) {
+        const int chunk = (c * 8 + f) ^ (r % NCH);
+        const float4 xr = *reinterpret_cast<const float4*>(sX + r * C::HALF + chunk * 4);
+        const float xs[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float val = fmaf(__uint_as_float(ov[4 * f + e]), inv, xs[e]);
+          y[32 * c + 4 * f + e] = val;
+          ss = fmaf(val, val, ss);
+        }
+      }
+    }
+    st_cluster_f32(map_to_cta(smem_u32(ssx + r), rank ^ 1u), ss);
+  }
+  cluster_sync_all();  // partner's half of the sum of squares visible
+  if (is_sm && qrow < N) {
+    const float tot = ss + ssx[r];
+    const float rs = rsqrtf(tot / static_cast<float>(C::DV) + p.eps);
+    const float gsc = (1.0f - p.lambda_init) * rs;
+    __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * N + qrow) * p.H + h) * C::DV + own0;
+#pragma unroll
+    for (int c8 = 0; c8 < C::HALF / 8; ++c8) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = 8 * c8 + 2 * e;
+        w4[e] = pack_bf16x2(y[c] * gsc * __ldg(p.rms_w + own0 + c), y[c + 1] * gsc * __ldg(p.rms_w + own0 + c + 1));
+      }
+      *reinterpret_cast<uint4*>(orow + 8 * c8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+template <int D>
+static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const PrefillParams& prm, int B, cudaStream_t stream) {
+  using C = Cfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * prm.n_qtiles, prm.H, B);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D>, tq, tk, tv, prm);
+}
+
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                                 int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
+                                 const float* rms_w, float eps, DevCtl ctl, cudaStream_t stream) {
+  PrefillParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.N = N;
+  prm.H = H;
+  prm.causal = causal ? 1 : 0;
+  prm.n_qtiles = (N + kBM - 1) / kBM;
+  prm.lambda = lambda;
+  prm.lambda_init = lambda_init;
+  prm.rms_w = rms_w;
+  prm.eps = eps;
+  prm.status = ctl.status;
+  prm.limit_ns = ctl.limit_ns;
+  if (d == 128) return launch_d<128>(tq, tk, tv, prm, B, stream);
+  if (d == 64) return launch_d<64>(tq, tk, tv, prm, B, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace diffattn

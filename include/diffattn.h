@@ -1,0 +1,164 @@
+/*
+ * diffattn.h -- C ABI of the differential-attention forward library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (page "Differential Transformer: Canceling Context Noise with
+ * Differential Attention", section "Cancelling Context Noise Through Attention
+ * Map Subtraction"; page "Differential attention", section "The
+ * noise-canceling idea"; peer review "Differential Transformer", Summary,
+ * Eqs. 1-3):
+ *
+ *   lambda   = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init            (Eq. 2)
+ *   O        = (softmax(Q1 K1^T / sqrt(d)) - lambda softmax(Q2 K2^T / sqrt(d))) V
+ *                                                                      (Eq. 1)
+ *   Y        = (1 - lambda_init) * w * O / sqrt(mean_c(O^2) + eps)     (Eq. 3)
+ *
+ * per head, where each head's query and key are split into two halves of
+ * width d (Q1|Q2, K1|K2) and V has width 2d (peer review, Strengths: heads are
+ * halved, h = d_model / 2d; Weaknesses: query/key width d, value width 2d).
+ * The headwise norm is RMSNorm over the 2d channels of each (token, head),
+ * eps inside the square root, with one weight vector w[2d] shared by all
+ * heads.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or keeps them.  The library allocates no device memory: the
+ *    decode path takes a caller-provided workspace.
+ *  - Every call is asynchronous and ordered on `stream` (0 = legacy default
+ *    stream).  The return value reports argument validation and launch
+ *    errors only; nothing is synchronised.  A kernel-side failure (a bounded
+ *    wait that ran out) is recorded in a device status word that
+ *    diffattn_device_status() reads.
+ *  - Tensors are dense and row-major in the layouts given below; every
+ *    tensor pointer must be 16-byte aligned.
+ *  - Return values are diffattn_status codes; 0 is success.
+ */
+#ifndef DIFFATTN_H_
+#define DIFFATTN_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DIFFATTN_OK = 0,
+  DIFFATTN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment      */
+  DIFFATTN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, d)      */
+  DIFFATTN_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed         */
+  DIFFATTN_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out           */
+  DIFFATTN_ERR_WORKSPACE = 5     /* workspace missing or too small            */
+} diffattn_status;
+
+typedef enum {
+  DIFFATTN_F32 = 0,   /* float32 storage and arithmetic                         */
+  DIFFATTN_BF16 = 1   /* bfloat16 storage, float32 accumulation                 */
+} diffattn_dtype;
+
+/*
+ * diffattn_lambda -- the lambda re-parameterisation (Eq. 2).
+ *
+ *   *lambda_out = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init
+ *
+ * lq1, lk1, lq2, lk2 : device float32[d], 1 <= d <= 4096.
+ * lambda_out         : device float32 scalar, written by the kernel.  The
+ *                      prefill and decode calls read lambda from this pointer,
+ *                      so no host round trip is needed.
+ * Errors: DIFFATTN_ERR_INVALID_ARG for a null pointer or d out of range.
+ */
+int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2,
+                    const float* lk2, int d, float lambda_init,
+                    float* lambda_out, cudaStream_t stream);
+
+/*
+ * diffattn_fwd -- prefill: differential attention for B sequences of N tokens
+ * followed by the headwise RMSNorm and the (1 - lambda_init) scale.
+ *
+ * q, k   : [B, N, H, 2, d]  (per head: Q1 then Q2, K1 then K2 -- the paper's
+ *                            2H heads of width d, in the same memory)
+ * v      : [B, N, H, 2d]
+ * o      : [B, N, H, 2d]    output, same dtype as the inputs
+ * dtype  : DIFFATTN_BF16 (tensor-core path; d must be 64 or 128) or
+ *          DIFFATTN_F32 (CUDA-core path; 1 <= d <= 128)
+ * causal : nonzero -> key j is visible to query i iff j <= i
+ * lambda : device float32 scalar (e.g. written by diffattn_lambda)
+ * rms_w  : device float32[2d], shared by all heads
+ * eps    : RMSNorm epsilon, >= 0, added to mean(O^2) inside the square root
+ *
+ * Sizes: B, H >= 1; N >= 0 (N = 0 is a no-op).  Shapes must satisfy
+ * B*N*H*2d < 2^31 elements per tensor and N < 2^31.
+ * Errors: DIFFATTN_ERR_INVALID_ARG (null/misaligned pointer, bad size),
+ * DIFFATTN_ERR_UNSUPPORTED (dtype/d combination), DIFFATTN_ERR_CUDA.
+ */
+int diffattn_fwd(const void* q, const void* k, const void* v, void* o,
+                 int dtype, int B, int N, int H, int d, int causal,
+                 const float* lambda, float lambda_init, const float* rms_w,
+                 float eps, cudaStream_t stream);
+
+/*
+ * diffattn_decode_workspace_size -- bytes of device workspace that
+ * diffattn_decode needs for S sequences of at most max_seqlen cached keys.
+ * Returns 0 for invalid sizes.
+ */
+size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen);
+
+/*
+ * diffattn_decode -- one decode step (query length 1) for S sequences over a
+ * packed KV cache, with the same DiffAttn + RMSNorm + scale as diffattn_fwd.
+ *
+ * q          : [S, H, 2, d] bf16 (Q1 then Q2 per head)
+ * k_cache    : [T, H, 2, d] bf16, sequences packed back to back
+ * v_cache    : [T, H, 2d]   bf16
+ * cu_seqlens : device int32[S + 1], cu_seqlens[0] = 0, non-decreasing;
+ *              sequence s owns cache rows cu_seqlens[s] .. cu_seqlens[s+1]-1
+ *              (its current token included) and its query sees all of them.
+ *              Every length must be in [1, max_seqlen].
+ * max_seqlen : host int, an upper bound on every sequence length
+ * o          : [S, H, 2d] bf16 output
+ * lambda, lambda_init, rms_w, eps : as in diffattn_fwd
+ * workspace  : device buffer of >= diffattn_decode_workspace_size() bytes,
+ *              16-byte aligned; its contents need no initialisation and
+ *              are scratch after the call.  Two calls that overlap on the
+ *              GPU must not share a workspace.
+ * Supported: d = 128, bf16 only (DIFFATTN_ERR_UNSUPPORTED otherwise).
+ * Errors: DIFFATTN_ERR_INVALID_ARG, DIFFATTN_ERR_WORKSPACE,
+ * DIFFATTN_ERR_CUDA.  A length outside [1, max_seqlen] is not detected on
+ * the host (cu_seqlens lives on the device): the kernel skips keys beyond
+ * max_seqlen and writes NaN for an empty sequence.
+ */
+int diffattn_decode(const void* q, const void* k_cache, const void* v_cache,
+                    const int* cu_seqlens, int max_seqlen, void* o, int S,
+                    int H, int d, const float* lambda, float lambda_init,
+                    const float* rms_w, float eps, void* workspace,
+                    size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * diffattn_device_status -- synchronises the current device, then returns
+ * the device-side status word (DIFFATTN_OK or DIFFATTN_ERR_TIMEOUT) in
+ * *status_out and clears it.  Returns DIFFATTN_ERR_CUDA if the device could
+ * not be queried.
+ */
+int diffattn_device_status(int* status_out);
+
+/*
+ * diffattn_set_wait_limit_ns -- upper bound, in nanoseconds, on every
+ * pipeline wait inside the library's kernels (default 2e9, i.e. 2 s; 0
+ * restores the default).  When a wait runs out, the kernel records
+ * DIFFATTN_ERR_TIMEOUT in the device status word, stops its pipeline,
+ * releases its tensor memory and returns, leaving the context usable.
+ * Applies to launches made after the call.
+ */
+int diffattn_set_wait_limit_ns(long long limit_ns);
+
+/* Human-readable name of a diffattn_status code. */
+const char* diffattn_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int diffattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DIFFATTN_H_ */

@@ -1,0 +1,89 @@
+"""The C-ABI library loads and exports every entry point declared in
+include/*.h; host-side validation rejects bad arguments before any CUDA call
+(no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from differential_attention_04_b200 import _lib, api
+from differential_attention_04_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        names |= set(re.findall(r"\b(diffattn_\w+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared()
+    assert {"diffattn_lambda", "diffattn_fwd", "diffattn_decode"} <= declared
+    for name in sorted(declared):
+        assert hasattr(L, name), f"{name} declared in include/ but not exported"
+
+
+def test_binding_covers_header(L):
+    assert _declared() == set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version(L):
+    assert L.diffattn_version() >= 100
+    for code in range(6):
+        assert L.diffattn_status_string(code)
+    assert L.diffattn_status_string(99) == b"unknown status"
+
+
+def test_validation_without_gpu(L):
+    # every case below is rejected before the library touches CUDA
+    nul = None
+    assert L.diffattn_lambda(nul, nul, nul, nul, 64, 0.5, nul, nul) == api.ERR_INVALID_ARG
+    fake = ctypes.c_void_p(4096)
+    assert L.diffattn_lambda(fake, fake, fake, fake, 0, 0.5, fake, nul) == api.ERR_INVALID_ARG
+    # prefill: bad sizes, bad dtype, null and misaligned pointers
+    args = lambda q, dt, B, N, H, d, eps=1e-5: L.diffattn_fwd(q, q, q, q, dt, B, N, H, d, 1, q, 0.5, q, eps, nul)
+    assert args(fake, api.BF16, 0, 16, 2, 128) == api.ERR_INVALID_ARG
+    assert args(fake, api.BF16, 1, -1, 2, 128) == api.ERR_INVALID_ARG
+    assert args(fake, 7, 1, 16, 2, 128) == api.ERR_INVALID_ARG
+    assert args(fake, api.BF16, 1, 16, 2, 128, eps=-1.0) == api.ERR_INVALID_ARG
+    assert args(nul, api.BF16, 1, 16, 2, 128) == api.ERR_INVALID_ARG
+    assert args(ctypes.c_void_p(4100), api.BF16, 1, 16, 2, 128) == api.ERR_INVALID_ARG
+    assert args(fake, api.BF16, 1, 16, 2, 96) == api.ERR_UNSUPPORTED
+    assert args(fake, api.F32, 1, 16, 2, 129) == api.ERR_UNSUPPORTED
+    assert args(fake, api.BF16, 1 << 16, 1 << 16, 2, 128) == api.ERR_INVALID_ARG  # > 2^31 elements
+    assert args(nul, api.BF16, 1, 0, 2, 128) == api.OK  # N = 0 is a no-op
+    # decode
+    dec = lambda q, d, ws, wsb, S=4: L.diffattn_decode(q, q, q, q, 100, q, S, 2, d, q, 0.5, q, 1e-5, ws, wsb, nul)
+    assert dec(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG
+    assert dec(fake, 64, fake, 1 << 30) == api.ERR_UNSUPPORTED
+    assert dec(fake, 128, nul, 1 << 30) == api.ERR_WORKSPACE
+    assert dec(fake, 128, fake, 16) == api.ERR_WORKSPACE
+    assert dec(fake, 128, fake, 1 << 30, S=0) == api.ERR_INVALID_ARG
+
+
+def test_workspace_size(L):
+    assert L.diffattn_decode_workspace_size(0, 12, 128, 100) == 0
+    assert L.diffattn_decode_workspace_size(4, 12, 64, 100) == 0
+    one = L.diffattn_decode_workspace_size(1, 1, 128, 1)
+    assert one > 0 and one % 16 == 0
+    # grows with the number of key chunks per sequence and with S * H
+    assert L.diffattn_decode_workspace_size(3, 5, 128, 1) == 15 * one
+    assert L.diffattn_decode_workspace_size(1, 1, 128, 100000) > one
+
+
+def test_wait_limit_setter(L):
+    assert L.diffattn_set_wait_limit_ns(-1) == api.ERR_INVALID_ARG
+    assert L.diffattn_set_wait_limit_ns(0) == api.OK

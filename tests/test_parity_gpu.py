@@ -138,8 +138,9 @@ def test_bf16_lambda_range(e1, e2, lambda_init, want):
     inp.lq2.fill_(math.sqrt(math.log(e2) / d))
     inp.lk2.copy_(inp.lq2)
     y, lam = run_prefill(inp)
-    assert abs(oracle_lambda(inp) - want) < 1e-12
-    assert abs(lam.item() - want) <= 1e-5
+    # the float32 lambda vectors hold ln(e)/d only to float32 precision
+    assert abs(oracle_lambda(inp) - want) < 1e-6
+    assert abs(lam.item() - oracle_lambda(inp)) <= 1e-6 * max(1.0, abs(want))
     assert_close(wl.to_f64(y), oracle_prefill(inp))
 
 

@@ -1,0 +1,65 @@
+"""Run one prefill or decode case a few times (e.g. under a profiler).
+
+  python -m differential_attention_04_b200.run_case prefill --B 2 --N 4096 --H 12 --d 128 --causal 1 --iters 3
+  python -m differential_attention_04_b200.run_case decode --S 64 --H 12 --lmin 1024 --lmax 4096 --iters 3
+
+Inputs come from the seeded generators in ``workloads``; the output is not
+checked here (the tests do that).  Prints the CUDA-event time of each launch.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import api
+from . import workloads as wl
+from .build import build
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kind", choices=["prefill", "decode"])
+    ap.add_argument("--B", type=int, default=2)
+    ap.add_argument("--N", type=int, default=4096)
+    ap.add_argument("--H", type=int, default=12)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--causal", type=int, default=1)
+    ap.add_argument("--dtype", default="bf16")
+    ap.add_argument("--S", type=int, default=64)
+    ap.add_argument("--lmin", type=int, default=1024)
+    ap.add_argument("--lmax", type=int, default=4096)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--seed", type=int, default=0)
+    a = ap.parse_args(argv)
+    build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if a.kind == "prefill":
+        inp = wl.make_prefill(a.B, a.N, a.H, a.d, causal=bool(a.causal), dtype=a.dtype, seed=a.seed, device=dev)
+        lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+        y = torch.empty_like(inp.v)
+        run = lambda: api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
+                                       out=y)
+    else:
+        inp = wl.make_decode(a.S, a.H, a.d, a.lmin, a.lmax, seed=a.seed, device=dev)
+        lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+        ws = torch.empty(api.decode_workspace_size(a.S, a.H, a.d, inp.max_seqlen), dtype=torch.uint8, device=dev)
+        y = torch.empty((a.S, a.H, 2 * a.d), dtype=torch.bfloat16, device=dev)
+        run = lambda: api.diffattn_decode(inp.q, inp.k_cache, inp.v_cache, inp.cu_seqlens, inp.max_seqlen, lam,
+                                          inp.lambda_init, inp.rms_w, inp.eps, workspace=ws, out=y)
+    torch.cuda.synchronize()
+    for i in range(a.iters):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        run()
+        e.record()
+        torch.cuda.synchronize()
+        print(f"{a.kind} iter {i}: {s.elapsed_time(e):.3f} ms")
+    status = api.device_status()
+    if status != api.OK:
+        raise SystemExit(f"kernel status {status}")
+
+
+if __name__ == "__main__":
+    main()

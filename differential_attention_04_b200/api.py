@@ -107,6 +107,30 @@ def diffattn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
     return out
 
 
+NOALLOC_SCRATCH_BYTES = 16 << 20  # DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES
+
+
+def diffattn_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                            cu_seqlens: torch.Tensor, max_seqlen: int, lam: torch.Tensor, lambda_init: float,
+                            rms_w: torch.Tensor, eps: float = 1e-5, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode without a workspace, for callers that may not allocate device memory.
+
+    The library's built-in 16 MiB device scratch replaces the workspace; calls
+    that overlap on the GPU share it and race.  Pass ``out`` to keep this call
+    free of allocations on the Python side as well.
+    """
+    _dev(q, k_cache, v_cache, cu_seqlens, lam, rms_w)
+    S, H, two, d = q.shape
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.numel() != S + 1:
+        raise ValueError("cu_seqlens must be int32 with S + 1 entries")
+    if out is None:
+        out = torch.empty((S, H, 2 * d), dtype=q.dtype, device=q.device)
+    _check("diffattn_decode_noalloc", lib().diffattn_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
+        _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _stream()))
+    return out
+
+
 def device_status() -> int:
     """Synchronise the device and return (and clear) the kernels' status word."""
     v = ctypes.c_int(0)

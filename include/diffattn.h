@@ -135,6 +135,43 @@ int diffattn_decode(const void* q, const void* k_cache, const void* v_cache,
                     size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * diffattn_decode_noalloc -- diffattn_decode for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a
+ * deployment variant of the same computation, with the same arguments as
+ * diffattn_decode except the workspace.
+ *
+ * Who needs it: callers that are not allowed to call cudaMalloc, for example
+ * a plugin inside an inference engine that owns all device memory through
+ * its own pool, or a serving loop that must never enter the driver's
+ * allocator.  They cannot hand diffattn_decode a workspace, so this call
+ * uses a scratch array that the library defines in device memory
+ * (DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES = 16 MiB).  The call itself
+ * allocates nothing.  Every GPU that loads the library holds that array
+ * until the process exits.
+ *
+ *  - Limit: problems with diffattn_decode_workspace_size(S, H, d,
+ *    max_seqlen) > DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES are rejected with
+ *    DIFFATTN_ERR_WORKSPACE before anything is launched (for example
+ *    S * H * ceil(max_seqlen / 512) must stay <= 8128 at d = 128).
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current).  Make that
+ *    first call before any stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    last call's contents.  Two calls that overlap on the GPU (on different
+ *    streams, or from different host threads) race on it; the caller must
+ *    order them.  Nothing needs clearing between calls: the kernels write
+ *    every scratch entry before they read it.
+ * Other errors as diffattn_decode.
+ */
+#define DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int diffattn_decode_noalloc(const void* q, const void* k_cache,
+                            const void* v_cache, const int* cu_seqlens,
+                            int max_seqlen, void* o, int S, int H, int d,
+                            const float* lambda, float lambda_init,
+                            const float* rms_w, float eps,
+                            cudaStream_t stream);
+
+/*
  * diffattn_device_status -- synchronises the current device, then returns
  * the device-side status word (DIFFATTN_OK or DIFFATTN_ERR_TIMEOUT) in
  * *status_out and clears it.  Returns DIFFATTN_ERR_CUDA if the device could

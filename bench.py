@@ -61,6 +61,28 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """Largest value of x over all ranks (the job's time is its slowest rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job rate: every rank processes its own batch (weak scaling); the
+    job takes as long as its slowest rank."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each replica draws its own seeded batch."""
+    return base + rank
+
+
 def prefill_flops(B, N, H, d, causal, convention):
     per_head = (16.0 if convention == "metric" else 12.0) * N * N * d
     return per_head * B * H * (0.5 if causal else 1.0)
@@ -267,15 +289,11 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def reduce_max(x: float) -> float:
+        return max_over_ranks(x, dist if world > 1 else None, dev)
 
     peaks, peak_src = load_peaks()
-    inp = wl.make_prefill_case(args.workload, seed=1234 + rank, device=dev)
+    inp = wl.make_prefill_case(args.workload, seed=rank_seed(1234, rank), device=dev)
     B, N, H, _, d = inp.q.shape
     lam = torch.empty(1, dtype=torch.float32, device=dev)
     y = torch.empty_like(inp.v)
@@ -306,7 +324,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_total = reduce_max(t0.elapsed_time(t1))
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     status = api.device_status()
     if status != api.OK:
@@ -315,7 +333,7 @@ def run_ours(args):
     ms_step = ms_total / K
     flops_metric = prefill_flops(B, N, H, d, inp.causal, "metric")
     flops_alg = prefill_flops(B, N, H, d, inp.causal, "algorithmic")
-    value = world * flops_metric / (ms_step * 1e-3) / 1e12
+    value = job_throughput(flops_metric, world, ms_step) / 1e12
     achieved = flops_alg / (kern_ms * 1e-3) / 1e12
     traffic = read_profile_traffic("prefill_sm100_prefill_3b")
 
@@ -344,8 +362,8 @@ def run_ours(args):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / E
-    e2e_value = world * flops_metric / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = reduce_max(e0.elapsed_time(e1)) / E
+    e2e_value = job_throughput(flops_metric, world, e2e_ms) / 1e12
     del dbuf, host, y_host
 
     line = {
@@ -373,7 +391,7 @@ def run_ours(args):
     }
 
     if not args.no_decode:
-        line["decode"] = bench_decode(api, wl, dev, peaks, peak_src, rank, max_over_ranks, barrier, world)
+        line["decode"] = bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world)
     del inp, y
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_inp = wl.make_prefill_case(args.workload, seed=1234, device="cpu")
@@ -386,10 +404,10 @@ def run_ours(args):
     return 0
 
 
-def bench_decode(api, wl, dev, peaks, peak_src, rank, max_over_ranks, barrier, world, steps=20):
+def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world, steps=20):
     import torch
 
-    inp = wl.make_decode_case(DECODE_WORKLOAD, seed=4321 + rank, device=dev)
+    inp = wl.make_decode_case(DECODE_WORKLOAD, seed=rank_seed(4321, rank), device=dev)
     S, H, _, d = inp.q.shape
     T = int(inp.seqlens.sum())
     lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
@@ -410,14 +428,14 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, max_over_ranks, barrier, w
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = max_over_ranks(a.elapsed_time(b)) / steps
+    ms = reduce_max(a.elapsed_time(b)) / steps
     kv_bytes = T * H * (2 * d + 2 * d) * 2
     io_bytes = S * H * 2 * d * 2 * 2
     alg = kv_bytes + io_bytes
     gbs = alg / (ms * 1e-3) / 1e9
     traffic = read_profile_traffic("decode_decode_64x12")
     return {
-        "metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+        "metric": "decode HBM GB/s", "value": job_throughput(alg, world, ms) / 1e9, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
         "workload": f"{DECODE_WORKLOAD}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
                     f"({kv_bytes / 1e9:.2f} GB per step)",
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

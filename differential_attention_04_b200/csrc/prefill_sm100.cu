@@ -13,9 +13,10 @@
 //   CTA rank i computes map i+1 only: S_i = Q_i K_i^T on the tensor cores,
 //   its own online softmax (running max m_i and sum l_i per row), and
 //   O_i += P_i V.  Both CTAs stream the same V tiles.  Tensor memory per CTA
-//   (512 columns): S double-buffered in columns [0,128) and [128,256), O_i in
-//   [256, 256 + 2d).  P (bf16) overwrites the upper 64 columns of its S
-//   buffer and feeds the PV product straight from tensor memory.
+//   (512 columns): S (fp32, one buffer) in columns [0, 128), P (bf16, two
+//   buffers of 64 columns) in [128, 256), O_i in [256, 256 + 2d).  P feeds
+//   the PV product straight from tensor memory.  Keeping P apart from S lets
+//   S_{j+1} be computed as soon as the softmax has read S_j into registers.
 //   The epilogue exchanges half of the columns through distributed shared
 //   memory: rank 0 keeps output columns [0, d), rank 1 keeps [d, 2d); each
 //   sends the other half of its O_i/l_i (scaled by -lambda on rank 1), the
@@ -28,15 +29,19 @@
 //   warp 3: idle                              warps 4-7: softmax + epilogue,
 //                                             one query row per thread
 //
-// Pipeline per key tile j (buffer b = j % 2):
-//   MMA:     S_j (keys 0-63 and 64-127 as two N=64 halves once the ring is
-//            warm) -> commit s_full[b]; wait p_full[b]; O += P_j V_j ->
-//            commit o_ready, v_empty.  The second half of S_{j+2} is issued
-//            only after PV_j has completed, because it overwrites P_j.
-//   softmax: wait s_full[b]; read the 128 scores of its row; mask; lazy
-//            rescale (O is rescaled only when the running max grows by more
-//            than 2^8, after PV_{j-1} has completed); P = exp2(s*c - m);
-//            store P as bf16 into tensor memory; arrive p_full[b].
+// Pipeline per key tile j (P buffer and K/V stage b = j % 2).  A
+// tcgen05.mma issue returns only when the instruction is nearly done, so the
+// issue order decides what overlaps:
+//   MMA:     wait s_free (the softmax has read S_{j-1}) -> S_j -> commit
+//            s_full, k_empty; then wait p_full[b'] of tile j-1 ->
+//            O += P_{j-1} V_{j-1} -> commit v_empty, p_empty[b'].  PV_{j-1}
+//            thus runs while the softmax works on tile j, and S_{j+1} is
+//            ready when the softmax finishes it.
+//   softmax: wait s_full; read the 128 scores of its row; arrive s_free;
+//            mask; lazy rescale (O is rescaled only when the running max
+//            grows by more than 2^8, after PV_{j-1} has completed); wait
+//            p_empty[b] (PV_{j-2} done); P = exp2(s*c - m) as bf16 into P[b];
+//            arrive p_full[b].
 #include <math.h>
 
 #include "common.cuh"
@@ -69,7 +74,8 @@ struct Cfg {
   static constexpr int OFF_SSX = OFF_BAR + 256;  // float[128]: partner's sum of squares
   static constexpr int SMEM_USED = OFF_SSX + 512;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
-  static constexpr uint32_t TM_S = 0;            // S buffer b at column 128 * b
+  static constexpr uint32_t TM_S = 0;            // S (fp32, 128 columns)
+  static constexpr uint32_t TM_P = 128;          // P buffer b (bf16 pairs) at column TM_P + 64 * b
   static constexpr uint32_t TM_O = 256;
   static constexpr uint32_t TM_COLS = 512;
   static_assert(kBM * HALF * 4 <= V_BYTES, "exchange buffer must fit in one V stage");
@@ -79,8 +85,8 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_ready;
+  uint64_t s_full, s_free;
+  uint64_t p_full[2], p_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -137,10 +143,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->k_empty[i], 1);
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->p_full[i], 4);  // one arrival per softmax warp
+      mbar_init(&bars->p_empty[i], 1);
     }
-    mbar_init(&bars->o_ready, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 4);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbarrier_init();
@@ -208,56 +215,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idesc_s128 = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_s64 = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      // S_buf[n_lo, n_lo + n_cnt) = Q K[n_lo : n_lo + n_cnt]^T for the K tile in stage `st`
-      auto issue_s = [&](int st, int buf, int n_lo, bool full) {
-        const uint32_t d_tmem = tmem + C::TM_S + 128 * buf + n_lo;
+      // O += P_t V_t, with P from buffer t % 2 and V from stage t % 2
+      auto issue_pv = [&](int t) -> bool {
+        const int bb = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!mbar_wait(&bars->v_full[bb], ph, wc)) return false;
+        if (!mbar_wait(&bars->p_full[bb], ph, wc)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t a_tmem = tmem + C::TM_P + 64 * bb + 8 * kk;
+          const uint64_t bd = smem_desc_sw128(sVa + bb * C::V_BYTES + kk * 2048, C::BLK_BYTES, 1024);
+          umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->v_empty[bb]);
+        umma_commit(&bars->p_empty[bb]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, wc);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int st = j & 1;
+        // S_j overwrites S_{j-1}: every softmax warp must have read it
+        if (j > 0 && !(ok = mbar_wait(&bars->s_free, (j - 1) & 1, wc))) break;
+        if (!(ok = mbar_wait(&bars->k_full[st], (j >> 1) & 1, wc))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int blk = kk >> 2;
           const uint32_t koff = (kk & 3) * 32;
           const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
-          const uint64_t bd =
-              smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + n_lo * 128 + koff, 16, 1024);
-          umma_ss(d_tmem, ad, bd, full ? idesc_s128 : idesc_s64, kk > 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + koff, 16, 1024);
+          umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-      };
-      bool ok = mbar_wait(&bars->q_full, 0, wc);
-      for (int t = 0; ok && t < min(2, n_kv); ++t) {
-        if (!(ok = mbar_wait(&bars->k_full[t], 0, wc))) break;
-        tc_fence_after();
-        issue_s(t, t, 0, true);
-        umma_commit(&bars->k_empty[t]);
-        umma_commit(&bars->s_full[t]);
+        umma_commit(&bars->k_empty[st]);
+        umma_commit(&bars->s_full);
+        if (j > 0) ok = issue_pv(j - 1);
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int bb = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!(ok = mbar_wait(&bars->v_full[bb], ph, wc))) break;
-        if (!(ok = mbar_wait(&bars->p_full[bb], ph, wc))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t a_tmem = tmem + C::TM_S + 128 * bb + 64 + 8 * kk;
-          const uint64_t bd = smem_desc_sw128(sVa + bb * C::V_BYTES + kk * 2048, C::BLK_BYTES, 1024);
-          umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->v_empty[bb]);
-        umma_commit(&bars->o_ready);
-        if (j + 2 < n_kv) {
-          if (!(ok = mbar_wait(&bars->k_full[bb], ((j + 2) >> 1) & 1, wc))) break;
-          tc_fence_after();
-          issue_s(bb, bb, 0, false);  // keys 0-63: columns already consumed by the softmax
-          if (!(ok = mbar_wait(&bars->o_ready, j & 1, wc))) break;  // PV_j done: P_j is free
-          tc_fence_after();
-          issue_s(bb, bb, 64, false);  // keys 64-127 overwrite P_j
-          umma_commit(&bars->k_empty[bb]);
-          umma_commit(&bars->s_full[bb]);
-        }
-      }
+      if (ok) issue_pv(n_kv - 1);
       // drain: every issued MMA has completed before tensor memory is read or freed
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, wdrain);
@@ -278,15 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n_kv; ++j) {
       const int bb = j & 1;
       const uint32_t ph = (j >> 1) & 1;
-      if (!(sm_ok = mbar_wait(&bars->s_full[bb], ph, wc))) break;
+      if (!(sm_ok = mbar_wait(&bars->s_full, j & 1, wc))) break;
       tc_fence_after();
       uint32_t s0[32], s1[32], s2[32], s3[32];
-      const uint32_t sb = tl + C::TM_S + 128 * bb;
+      const uint32_t sb = tl + C::TM_S;
       tmem_ld32(sb + 0, s0);
       tmem_ld32(sb + 32, s1);
       tmem_ld32(sb + 64, s2);
       tmem_ld32(sb + 96, s3);
       tmem_ld_wait4(s0, s1, s2, s3);
+      // S is in registers: the next S tile may overwrite the buffer
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free);
       float x[128];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -302,9 +303,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 128; ++i)
           if (key0 + i > lim) x[i] = -INFINITY;
       }
-      float mx = x[0];
+      // row maximum with eight independent chains (short dependency depth)
+      float mk[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, x[i]);
+      for (int c = 0; c < 8; ++c) mk[c] = x[c];
+#pragma unroll
+      for (int i = 8; i < 128; i += 8) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mk[c] = fmaxf(mk[c], x[i + c]);
+      }
+      const float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
+                             fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
       const float t_mx = mx * sc;
       if (j == 0) {
         m_run = t_mx;
@@ -312,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool need = t_mx > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? fast_exp2(m_run - t_mx) : 1.0f;
-          if (!(sm_ok = mbar_wait(&bars->o_ready, (j - 1) & 1, wc))) break;  // PV_{j-1} done
+          // O may be rescaled only once PV_{j-1} has completed
+          if (!(sm_ok = mbar_wait(&bars->p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wc))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < C::DV / 32; ++c) {
@@ -328,26 +338,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (need) m_run = t_mx;
         }
       }
+      // P_j reuses the buffer of P_{j-2}: PV_{j-2} must have completed
+      if (j >= 2 && !(sm_ok = mbar_wait(&bars->p_empty[bb], ph ^ 1u, wc))) break;
+      tc_fence_after();
       const float mneg = -m_run;
-      uint32_t pk[32];
-      float lsum = 0.f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t pb = tl + C::TM_P + 64 * bb;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float p0 = fast_exp2(fmaf(x[64 * half + 2 * i], sc, mneg));
           const float p1 = fast_exp2(fmaf(x[64 * half + 2 * i + 1], sc, mneg));
-          lsum += p0 + p1;
+          acc[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(sb + 64 + 32 * half, pk);
+        tmem_st32(pb + 32 * half, pk);
       }
       tmem_st_wait();
-      l_run += lsum;
+      l_run += (acc[0] + acc[1]) + (acc[2] + acc[3]);
       tc_fence_before();
-      mbar_arrive(&bars->p_full[bb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[bb]);
     }
-    if (sm_ok) sm_ok = mbar_wait(&bars->o_ready, (n_kv - 1) & 1, wc);  // last PV done
+    // O is complete once the last two PV products have (earlier ones were
+    // waited for above)
+    for (int t = max(0, n_kv - 2); sm_ok && t < n_kv; ++t)
+      sm_ok = mbar_wait(&bars->p_empty[t & 1], (t >> 1) & 1, wc);
     tc_fence_after();
   }
 

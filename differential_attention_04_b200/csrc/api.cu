@@ -138,16 +138,16 @@ int diffattn_fwd(const void* q, const void* k, const void* v, void* o, int dtype
                                                causal, lambda, lambda_init, rms_w, eps, stream));
   }
   if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
-      !encode_4d(&tv, v, 2ull * d, H, N, B))
+      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   cudaError_t e = status_ptr(&ctl.status);
   if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
   return cuda_status(
-      launch_prefill_sm100(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, ctl, stream));
+      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, ctl, stream));
 }
 
 size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen) {

@@ -376,6 +376,14 @@ __device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst_cluster, const 
       "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
       : "memory");
 }
+// 4-D tiled TMA store from this CTA's shared memory (bulk-group completion);
+// elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+               ::"l"(m), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the sources of this thread's bulk copies have been read.
 __device__ __forceinline__ void bulk_wait_group_read0() {

@@ -24,7 +24,8 @@ cudaError_t launch_prefill_simt_f32(const float* q, const float* k, const float*
 // Tensor-core (tcgen05) prefill for bf16 tensors, d in {64, 128}.  tq/tk map
 // [B, N, H*2, d]; tv maps [B, N, H, 2d]; boxes are 64 columns x 128 rows with
 // 128-byte swizzle.
-cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, DevCtl ctl, cudaStream_t stream);
 

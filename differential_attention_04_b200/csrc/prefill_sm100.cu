@@ -19,9 +19,10 @@
 //   S_{j+1} be computed as soon as the softmax has read S_j into registers.
 //   The epilogue exchanges half of the columns through distributed shared
 //   memory: rank 0 keeps output columns [0, d), rank 1 keeps [d, 2d); each
-//   sends the other half of its O_i/l_i (scaled by -lambda on rank 1), the
-//   two halves of the row's sum of squares are swapped, and each CTA writes
-//   its columns of (1 - lambda_init) * w * O / rms.
+//   bulk-copies the other half of its O_i/l_i (scaled by -lambda on rank 1)
+//   into the partner's shared memory, the partial sums of squares of each
+//   row are swapped, and each CTA stages its columns of
+//   (1 - lambda_init) * w * O / rms as bf16 and writes them with TMA stores.
 //
 // Warp roles (256 threads)
 //   warp 0: TMA producer for Q_i and K_i      warp 2: TMA producer for V
@@ -37,11 +38,14 @@
 //            O += P_{j-1} V_{j-1} -> commit v_empty, p_empty[b'].  PV_{j-1}
 //            thus runs while the softmax works on tile j, and S_{j+1} is
 //            ready when the softmax finishes it.
-//   softmax: wait s_full; read the 128 scores of its row; arrive s_free;
-//            mask; lazy rescale (O is rescaled only when the running max
-//            grows by more than 2^8, after PV_{j-1} has completed); wait
-//            p_empty[b] (PV_{j-2} done); P = exp2(s*c - m) as bf16 into P[b];
-//            arrive p_full[b].
+//   softmax: wait s_full (S_j done, and so every MMA issued before it:
+//            PV_{j-2}, the last reader of P[b]); read the 128 scores of its
+//            row; arrive s_free; mask; P = exp2(s*c - m) as bf16 into P[b],
+//            relative to the reference maximum m, while forming the tile's
+//            own maximum; arrive p_full[b].  Lazy rescale: only when the
+//            running maximum exceeds m by more than 2^8 are O and l rescaled
+//            to it, once PV_j has completed; a jump beyond 2^64, which could
+//            overflow P, rescales first and recomputes P.
 #include <math.h>
 
 #include "common.cuh"
@@ -56,6 +60,7 @@ constexpr int kBM = 128;  // query rows per CTA
 constexpr int kBN = 128;  // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kOverflowGuard = 64.0f;    // log2 units
 
 template <int D>
 struct Cfg {
@@ -71,14 +76,16 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + 2 * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + 2 * V_BYTES;
-  static constexpr int OFF_SSX = OFF_BAR + 256;  // float[128]: partner's sum of squares
-  static constexpr int SMEM_USED = OFF_SSX + 512;
+  static constexpr int SMEM_USED = OFF_BAR + 256;
+  static constexpr int EXCH_BYTES = kBM * HALF * 4;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
   static constexpr uint32_t TM_S = 0;            // S (fp32, 128 columns)
   static constexpr uint32_t TM_P = 128;          // P buffer b (bf16 pairs) at column TM_P + 64 * b
   static constexpr uint32_t TM_O = 256;
   static constexpr uint32_t TM_COLS = 512;
-  static_assert(kBM * HALF * 4 <= V_BYTES, "exchange buffer must fit in one V stage");
+  static_assert(EXCH_BYTES <= V_BYTES, "exchange buffers must fit in one V stage each");
+  static_assert(kBM * HALF * 2 <= 2 * K_BYTES, "output staging must fit in the K stages");
+
 };
 
 struct Bars {
@@ -88,6 +95,7 @@ struct Bars {
   uint64_t s_full, s_free;
   uint64_t p_full[2], p_empty[2];
   uint64_t mma_done;
+  uint64_t exch_full;  // the partner's half of the output has landed
   uint32_t tmem_base;
   int abort;
 };
@@ -117,7 +125,8 @@ __device__ __forceinline__ void tmem_ld_wait4(uint32_t (&a)[32], uint32_t (&b)[3
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                         const __grid_constant__ CUtensorMap tv, const PrefillParams p) {
+                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                         const PrefillParams p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,8 +134,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
-  float* ssx = reinterpret_cast<float*>(smem + C::OFF_SSX);
-  float* sX = reinterpret_cast<float*>(sV);  // epilogue exchange buffer (V stage 0)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();  // 0: map 1, 1: map 2
@@ -149,13 +156,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 4);
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->exch_full, 1);
     bars->abort = 0;
     fence_mbarrier_init();
+    mbar_arrive_expect_tx(&bars->exch_full, C::EXCH_BYTES);  // armed long before the partner sends
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&to);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, C::TM_COLS);
@@ -272,17 +282,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool sm_ok = true;
   if (is_sm) {
     const float sc = kLog2e * rsqrtf(static_cast<float>(D));
+    // O and l *= alpha (the whole warp takes part; alpha = 1 leaves a row as it is)
+    auto rescale_o = [&](float alpha) {
+#pragma unroll
+      for (int c = 0; c < C::DV / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32_sync(tl + C::TM_O + 32 * c, ov);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+        tmem_st32(tl + C::TM_O + 32 * c, ov);
+      }
+      tmem_st_wait();
+      l_run *= alpha;
+    };
     for (int j = 0; j < n_kv; ++j) {
       const int bb = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
       if (!(sm_ok = mbar_wait(&bars->s_full, j & 1, wc))) break;
+      // S_j has completed, and with it every MMA issued before it, PV_{j-2}
+      // included: P buffer b is free.
       tc_fence_after();
       uint32_t s0[32], s1[32], s2[32], s3[32];
-      const uint32_t sb = tl + C::TM_S;
-      tmem_ld32(sb + 0, s0);
-      tmem_ld32(sb + 32, s1);
-      tmem_ld32(sb + 64, s2);
-      tmem_ld32(sb + 96, s3);
+      tmem_ld32(tl + C::TM_S + 0, s0);
+      tmem_ld32(tl + C::TM_S + 32, s1);
+      tmem_ld32(tl + C::TM_S + 64, s2);
+      tmem_ld32(tl + C::TM_S + 96, s3);
       tmem_ld_wait4(s0, s1, s2, s3);
       // S is in registers: the next S tile may overwrite the buffer
       tc_fence_before();
@@ -298,113 +321,132 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int key0 = j * kBN;
       if (key0 + kBN > N || (p.causal && j == qtile)) {
-        const int lim = p.causal ? min(N - 1, qrow) : N - 1;  // last visible key
+        const int lim = (p.causal ? min(N - 1, qrow) : N - 1) - key0;  // last visible key of the tile
 #pragma unroll
         for (int i = 0; i < 128; ++i)
-          if (key0 + i > lim) x[i] = -INFINITY;
+          if (i > lim) x[i] = -INFINITY;
       }
-      // row maximum with eight independent chains (short dependency depth)
-      float mk[8];
+      if (j == 0) {  // the first tile sets the reference maximum
+        float mk[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mk[c] = x[c];
+        for (int c = 0; c < 8; ++c) mk[c] = x[c];
 #pragma unroll
-      for (int i = 8; i < 128; i += 8) {
+        for (int i = 8; i < 128; i += 8) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mk[c] = fmaxf(mk[c], x[i + c]);
+          for (int c = 0; c < 8; ++c) mk[c] = fmaxf(mk[c], x[i + c]);
+        }
+        m_run = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])), fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7]))) * sc;
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
-                             fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
-      const float t_mx = mx * sc;
-      if (j == 0) {
-        m_run = t_mx;
-      } else {
-        const bool need = t_mx > m_run + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? fast_exp2(m_run - t_mx) : 1.0f;
-          // O may be rescaled only once PV_{j-1} has completed
-          if (!(sm_ok = mbar_wait(&bars->p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wc))) break;
-          tc_fence_after();
+      // P = exp2(s*c - m_run) into P[b], taken relative to the reference
+      // maximum m_run as it stands; the tile's own maximum is formed alongside.
+      float lsum = 0.f, t_mx = -INFINITY;
+      auto make_p = [&](bool with_max) {
+        const float mneg = -m_run;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float mk[8];
 #pragma unroll
-          for (int c = 0; c < C::DV / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tl + C::TM_O + 32 * c, ov);
-            tmem_ld_wait(ov);
+        for (int c = 0; c < 8; ++c) mk[c] = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(tl + C::TM_O + 32 * c, ov);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float a0 = x[64 * half + 2 * i], a1 = x[64 * half + 2 * i + 1];
+            if (with_max) mk[i & 7] = fmaxf(mk[i & 7], fmaxf(a0, a1));
+            const float p0 = fast_exp2(fmaf(a0, sc, mneg));
+            const float p1 = fast_exp2(fmaf(a1, sc, mneg));
+            acc[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
           }
-          tmem_st_wait();
-          l_run *= alpha;
-          if (need) m_run = t_mx;
+          tmem_st32(tl + C::TM_P + 64 * bb + 32 * half, pk);
         }
-      }
-      // P_j reuses the buffer of P_{j-2}: PV_{j-2} must have completed
-      if (j >= 2 && !(sm_ok = mbar_wait(&bars->p_empty[bb], ph ^ 1u, wc))) break;
-      tc_fence_after();
-      const float mneg = -m_run;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t pb = tl + C::TM_P + 64 * bb;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = fast_exp2(fmaf(x[64 * half + 2 * i], sc, mneg));
-          const float p1 = fast_exp2(fmaf(x[64 * half + 2 * i + 1], sc, mneg));
-          acc[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(pb + 32 * half, pk);
+        lsum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        if (with_max)
+          t_mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])), fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7]))) * sc;
+      };
+      make_p(true);
+      // A jump of the maximum by more than 2^64 would overflow P: rescale O
+      // to the new maximum (after PV_{j-1} has completed) and redo P.
+      const bool hard = t_mx > m_run + kOverflowGuard;
+      if (__any_sync(0xffffffffu, hard)) {
+        tmem_st_wait();
+        if (!(sm_ok = mbar_wait(&bars->p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wc))) break;
+        tc_fence_after();
+        rescale_o(hard ? fast_exp2(m_run - t_mx) : 1.0f);
+        if (hard) m_run = t_mx;
+        make_p(false);
       }
       tmem_st_wait();
-      l_run += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      l_run += lsum;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[bb]);
+      // Lazy rescale: keep the reference within 2^8 of the running maximum.
+      // O is rescaled once PV_j (which used the old reference) has completed.
+      const bool need = t_mx > m_run + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, need)) {
+        if (!(sm_ok = mbar_wait(&bars->p_empty[bb], (j >> 1) & 1, wc))) break;
+        tc_fence_after();
+        rescale_o(need ? fast_exp2(m_run - t_mx) : 1.0f);
+        if (need) m_run = t_mx;
+      }
     }
-    // O is complete once the last two PV products have (earlier ones were
-    // waited for above)
-    for (int t = max(0, n_kv - 2); sm_ok && t < n_kv; ++t)
-      sm_ok = mbar_wait(&bars->p_empty[t & 1], (t >> 1) & 1, wc);
+    // O is complete once the last PV (and with it every earlier MMA) has
+    if (sm_ok) sm_ok = mbar_wait(&bars->p_empty[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, wc);
     tc_fence_after();
   }
 
   // ----------------------------------------------------------- epilogue --
-  cluster_sync_all();  // both CTAs: main loops drained, V stage 0 free for the exchange
+  // After the first cluster barrier every MMA and TMA load of both CTAs has
+  // completed, so Q, K and V space is reused: sums of squares in the Q tile,
+  // the partner's half in V stage 0, the half sent to it in V stage 1, the
+  // bf16 output tile in the K stages.
+  float* ssx = reinterpret_cast<float*>(sQ);  // [128] the partner's sums of squares, written remotely
+  float* recv = reinterpret_cast<float*>(sV);
+  float* stage = reinterpret_cast<float*>(sV + C::V_BYTES);
+  uint8_t* sOut = sK;
+  const uint32_t partner = rank ^ 1u;
+  constexpr int HALF = C::HALF;
+  constexpr int NC = HALF / 4;  // float4 chunks per exchanged row
+  cluster_sync_all();  // both CTAs: main loops drained, buffers free
   const float lam = *p.lambda;
-  const float inv = (rank == 0) ? 1.0f / l_run : -lam / l_run;
-  const int own0 = (rank == 0) ? 0 : C::HALF;   // columns this CTA finishes
-  const int send0 = (rank == 0) ? C::HALF : 0;  // columns the partner finishes
-  constexpr int NCH = C::HALF / 4;              // float4 chunks per exchange row
-  if (is_sm) {
-    const uint32_t remote = map_to_cta(smem_u32(sX), rank ^ 1u);
-#pragma unroll
-    for (int c = 0; c < C::HALF / 32; ++c) {
-      uint32_t ov[32];
-      tmem_ld32(tl + C::TM_O + send0 + 32 * c, ov);
-      tmem_ld_wait(ov);
-#pragma unroll
-      for (int f = 0; f < 8; ++f) {
-        const int chunk = (c * 8 + f) ^ (r % NCH);
-        st_cluster_v4(remote + static_cast<uint32_t>((r * C::HALF + chunk * 4) * 4),
-                      __uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
-                      __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
-      }
-    }
-  }
-  cluster_sync_all();  // exchanged halves visible
-  float y[C::HALF];
+  const int own0 = (rank == 0) ? 0 : HALF;   // columns this CTA finishes
+  const int send0 = (rank == 0) ? HALF : 0;  // columns it hands to the partner
+  float y[HALF];
   float ss = 0.f;
   if (is_sm) {
+    const float inv = (rank == 0) ? 1.0f / l_run : -lam / l_run;
+    float* srow = stage + r * HALF;
 #pragma unroll
-    for (int c = 0; c < C::HALF / 32; ++c) {
+    for (int c = 0; c < HALF / 32; ++c) {
       uint32_t ov[32];
-      tmem_ld32(tl + C::TM_O + own0 + 32 * c, ov);
-      tmem_ld_wait(ov);
+      tmem_ld32_sync(tl + C::TM_O + send0 + 32 * c, ov);
 #pragma unroll
       for (int f = 0; f < 8; ++f) {
-        const int chunk = (c * 8 + f) ^ (r % NCH);
-        const float4 xr = *reinterpret_cast<const float4*>(sX + r * C::HALF + chunk * 4);
+        const int chunk = (c * 8 + f) ^ (r % NC);
+        *reinterpret_cast<float4*>(srow + chunk * 4) =
+            make_float4(__uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                        __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
+      }
+    }
+    fence_proxy_async_smem();  // the staged rows are read by the bulk copy (async proxy)
+    __syncwarp();
+    if (lane == 0) {
+      const int off = quarter * 32 * HALF;  // this warp's 32 rows, contiguous
+      bulk_copy_s2cluster(map_to_cta(smem_u32(recv + off), partner), stage + off, 32 * HALF * 4,
+                          map_to_cta(smem_u32(&bars->exch_full), partner));
+      bulk_commit_group();
+    }
+    mbar_wait(&bars->exch_full, 0, wdrain);  // the partner's half has landed
+    const float* rrow = recv + r * HALF;
+#pragma unroll
+    for (int c = 0; c < HALF / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld32_sync(tl + C::TM_O + own0 + 32 * c, ov);
+#pragma unroll
+      for (int f = 0; f < 8; ++f) {
+        const int chunk = (c * 8 + f) ^ (r % NC);
+        const float4 xr = *reinterpret_cast<const float4*>(rrow + chunk * 4);
         const float xs[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -414,24 +456,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    st_cluster_f32(map_to_cta(smem_u32(ssx + r), rank ^ 1u), ss);
+    st_cluster_f32(map_to_cta(smem_u32(ssx + r), partner), ss);
+    if (lane == 0) bulk_wait_group_read0();  // the outgoing copy has left this CTA's memory
+    __syncwarp();
   }
-  cluster_sync_all();  // partner's half of the sum of squares visible
-  if (is_sm && qrow < N) {
-    const float tot = ss + ssx[r];
-    const float rs = rsqrtf(tot / static_cast<float>(C::DV) + p.eps);
+  cluster_sync_all();  // the partner's partial sums of squares visible; no remote access after this
+  if (is_sm) {
+    const float rs = rsqrtf((ss + ssx[r]) / static_cast<float>(C::DV) + p.eps);
     const float gsc = (1.0f - p.lambda_init) * rs;
-    __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * N + qrow) * p.H + h) * C::DV + own0;
+    // bf16 tile [64-column block][128 rows][64 columns], 128-byte swizzle
 #pragma unroll
-    for (int c8 = 0; c8 < C::HALF / 8; ++c8) {
+    for (int c8 = 0; c8 < HALF / 8; ++c8) {
       uint32_t w4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int c = 8 * c8 + 2 * e;
         w4[e] = pack_bf16x2(y[c] * gsc * __ldg(p.rms_w + own0 + c), y[c + 1] * gsc * __ldg(p.rms_w + own0 + c + 1));
       }
-      *reinterpret_cast<uint4*>(orow + 8 * c8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      const uint32_t a = smem_u32(sOut) + (c8 / 8) * C::BLK_BYTES + r * 128 + (((c8 % 8) ^ (r & 7)) << 4);
+      st_shared_v4(a, w4[0], w4[1], w4[2], w4[3]);
     }
+    fence_proxy_async_smem();  // the tile is read by the TMA store (async proxy)
+    named_bar_sync(1, 128);    // the four softmax warps have staged their rows
+    if (warp == 4 && lane == 0) {
+#pragma unroll
+      for (int blk = 0; blk < HALF / 64; ++blk)
+        tma_store_4d(&to, sOut + blk * C::BLK_BYTES, own0 + 64 * blk, h, qtile * kBM, b);  // rows >= N are clipped
+      bulk_commit_group();
+      bulk_wait_group_read0();  // shared memory must stay valid until the store has read it
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -443,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const PrefillParams& prm, int B, cudaStream_t stream) {
+                            const CUtensorMap& to, const PrefillParams& prm, int B, cudaStream_t stream) {
   using C = Cfg<D>;
   cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
@@ -460,10 +514,11 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D>, tq, tk, tv, prm);
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D>, tq, tk, tv, to, prm);
 }
 
-cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, DevCtl ctl, cudaStream_t stream) {
   PrefillParams prm;
@@ -478,8 +533,8 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.eps = eps;
   prm.status = ctl.status;
   prm.limit_ns = ctl.limit_ns;
-  if (d == 128) return launch_d<128>(tq, tk, tv, prm, B, stream);
-  if (d == 64) return launch_d<64>(tq, tk, tv, prm, B, stream);
+  if (d == 128) return launch_d<128>(tq, tk, tv, to, prm, B, stream);
+  if (d == 64) return launch_d<64>(tq, tk, tv, to, prm, B, stream);
   return cudaErrorInvalidValue;
 }
 

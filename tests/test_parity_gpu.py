@@ -163,6 +163,20 @@ def test_bf16_large_scores():
     assert_close(wl.to_f64(y), oracle_prefill(inp))
 
 
+def test_bf16_score_jumps():
+    # keys scaled up along the sequence: the running maximum climbs by far
+    # more than 2^64 (log2 units) between key tiles, which takes the
+    # overflow-guard path (rescale O first, then recompute P) as well as the
+    # lazy rescale after PV
+    inp = wl.make_prefill(1, 640, 2, 128, causal=True, dtype="bf16", lambda_init=0.5, seed=11, device="cuda")
+    ramp = torch.linspace(1.0, 24.0, 640, device="cuda").view(1, 640, 1, 1, 1)
+    inp.k.copy_((inp.k.float() * ramp).to(inp.k.dtype))
+    inp.q.mul_(4)
+    y, _ = run_prefill(inp)
+    assert torch.isfinite(y.float()).all()
+    assert_close(wl.to_f64(y), oracle_prefill(inp))
+
+
 def test_output_only_written_in_bounds():
     inp = wl.make_prefill(1, 200, 2, 128, causal=True, dtype="bf16", seed=3, device="cuda")
     lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)

@@ -50,7 +50,8 @@ invariant 1 - lambda, lambda = 0 against torch's scaled_dot_product_attention
 (a library routine), map 2 alone against the same routine, Q2=Q1/K2=K1 giving
 (1 - lambda) times single-map attention, the single visible key of causal row
 0, hand-computed RMSNorm and lambda values, brute-force loops on tiny shapes,
-and decode == last prefill row.
+decode == last prefill row, and for the two control modes (lambda = 0:
+one map; "+lambda": the maps added) torch's attention per map.
 """
 from __future__ import annotations
 
@@ -60,6 +61,8 @@ import numpy as np
 
 __all__ = [
     "lambda_reparam",
+    "MODES",
+    "map_weights",
     "softmax_rows",
     "diff_weights",
     "diffattn_head_prenorm",
@@ -109,6 +112,30 @@ def diff_weights(S1: np.ndarray, S2: np.ndarray, lam: float) -> np.ndarray:
     return softmax_rows(S1) - float(lam) * softmax_rows(S2)
 
 
+# Combination of the two maps, D = softmax(S1) + c * softmax(S2):
+#   "diff"        c = -lambda : the DiffAttn equation (the method itself)
+#   "lambda_zero" c = 0       : the peer review's lambda = 0 control (Questions,
+#                               first bullet; Weaknesses, second bullet): the same
+#                               architecture with a single softmax map
+#   "sum"         c = +lambda : the review's "+lambda" control, two maps added
+#                               rather than subtracted (same bullets)
+MODES = ("diff", "lambda_zero", "sum")
+
+
+def map_weights(S1: np.ndarray, S2: np.ndarray, lam: float, mode: str = "diff") -> np.ndarray:
+    """softmax(S1) + c * softmax(S2) with c given by ``mode`` (see MODES).
+
+    "lambda_zero" uses softmax(S1) alone (S2 is not looked at).
+    """
+    if mode == "diff":
+        return diff_weights(S1, S2, lam)
+    if mode == "lambda_zero":
+        return softmax_rows(S1)
+    if mode == "sum":
+        return softmax_rows(S1) + float(lam) * softmax_rows(S2)
+    raise ValueError(f"mode must be one of {MODES}")
+
+
 def _causal_scores(q: np.ndarray, k: np.ndarray, scale: float, q_pos, causal: bool) -> np.ndarray:
     """Scores q k^T * scale for the query positions ``q_pos`` against all keys.
 
@@ -123,7 +150,7 @@ def _causal_scores(q: np.ndarray, k: np.ndarray, scale: float, q_pos, causal: bo
     return S
 
 
-def diffattn_head_prenorm(q1, k1, q2, k2, v, lam: float, causal: bool, rows=None) -> np.ndarray:
+def diffattn_head_prenorm(q1, k1, q2, k2, v, lam: float, causal: bool, rows=None, mode: str = "diff") -> np.ndarray:
     """DiffAttn for one head, before the headwise norm.
 
     q1, q2 : [N, d]   k1, k2 : [N, d]   v : [N, 2d]   ->   O : [len(rows), 2d]
@@ -135,6 +162,7 @@ def diffattn_head_prenorm(q1, k1, q2, k2, v, lam: float, causal: bool, rows=None
     with Differential Attention", "Cancelling Context Noise Through Attention
     Map Subtraction"; peer review Eq. 1), with d = the per-map width (the
     peer review's lambda=0 control: query/key width d = 128, value width 2d).
+    ``mode`` selects the combination of the two maps (see MODES).
     """
     q1 = np.asarray(q1, dtype=np.float64)
     q2 = np.asarray(q2, dtype=np.float64)
@@ -148,7 +176,7 @@ def diffattn_head_prenorm(q1, k1, q2, k2, v, lam: float, causal: bool, rows=None
     scale = 1.0 / math.sqrt(d)
     S1 = _causal_scores(q1[rows], k1, scale, rows, causal)
     S2 = _causal_scores(q2[rows], k2, scale, rows, causal)
-    D = diff_weights(S1, S2, lam)
+    D = map_weights(S1, S2, lam, mode)
     return D @ v
 
 
@@ -167,12 +195,13 @@ def headwise_rmsnorm(O: np.ndarray, w, eps: float, lambda_init: float) -> np.nda
 
 
 def diffattn_fwd(q, k, v, lam: float, lambda_init: float, w, eps: float, causal: bool,
-                 rows=None, heads=None) -> np.ndarray:
+                 rows=None, heads=None, mode: str = "diff") -> np.ndarray:
     """Prefill: normalised DiffAttn output for every (batch, head).
 
     q, k : [B, N, H, 2, d]; v : [B, N, H, 2d].  Returns y : [B, R, H, 2d] where
     R = N, or the query positions in ``rows``.  ``heads`` (optional) is a list
-    of (b, h) pairs to compute; the others are left as NaN.
+    of (b, h) pairs to compute; the others are left as NaN.  ``mode`` selects
+    the combination of the two maps (see MODES).
     """
     q = np.asarray(q)
     k = np.asarray(k)
@@ -185,7 +214,7 @@ def diffattn_fwd(q, k, v, lam: float, lambda_init: float, w, eps: float, causal:
     for b, h in pairs:
         O = diffattn_head_prenorm(q[b, :, h, 0, :], k[b, :, h, 0, :],
                                   q[b, :, h, 1, :], k[b, :, h, 1, :],
-                                  v[b, :, h, :], lam, causal, rows)
+                                  v[b, :, h, :], lam, causal, rows, mode)
         y[b, :, h, :] = headwise_rmsnorm(O, w, eps, lambda_init)
     return y
 

@@ -228,9 +228,58 @@ def pin_sampled_rows():
         assert np.allclose(full[:, rows], part, atol=1e-13)
 
 
+def _hand_rmsnorm(O, w, eps, lambda_init):
+    out = np.empty_like(O)
+    for i in range(O.shape[0]):
+        ms = sum(float(x) * float(x) for x in O[i]) / O.shape[1]
+        out[i] = (1.0 - lambda_init) * w * O[i] / math.sqrt(ms + eps)
+    return out
+
+
+def pin_mode_lambda_zero():
+    # the review's lambda = 0 control: one softmax map (map 1), whatever map 2
+    # and lambda are; torch's attention on map 1, then the headwise norm
+    rng = np.random.default_rng(21)
+    n, d = 9, 4
+    q1, k1, q2, k2, v = _rand_head(rng, n, d)
+    w = 1 + 0.1 * rng.standard_normal(2 * d)
+    q = np.stack([q1, q2], 1)[None, :, None]
+    k = np.stack([k1, k2], 1)[None, :, None]
+    for causal in (False, True):
+        y = ref.diffattn_fwd(q, k, v[None, :, None], 0.7, 0.3, w, 1e-5, causal, mode="lambda_zero")[0, :, 0]
+        want = _hand_rmsnorm(_sdpa(q1, k1, v, causal), w, 1e-5, 0.3)
+        assert np.allclose(y, want, atol=1e-12)
+        q[0, :, 0, 1] = rng.standard_normal((n, d))  # map 2 changes: the output does not
+        y2 = ref.diffattn_fwd(q, k, v[None, :, None], -1.3, 0.3, w, 1e-5, causal, mode="lambda_zero")[0, :, 0]
+        assert np.array_equal(y, y2)
+
+
+def pin_mode_sum():
+    # the review's "+lambda" control: the two maps added; against torch's
+    # attention per map, the row sums 1 + lambda, and sum(lambda) = diff(-lambda)
+    rng = np.random.default_rng(22)
+    n, d = 10, 4
+    q1, k1, q2, k2, v = _rand_head(rng, n, d)
+    lam = 0.45
+    for causal in (False, True):
+        O = ref.diffattn_head_prenorm(q1, k1, q2, k2, v, lam, causal, mode="sum")
+        want = _sdpa(q1, k1, v, causal) + lam * _sdpa(q2, k2, v, causal)
+        assert np.allclose(O, want, atol=1e-12)
+        O_neg = ref.diffattn_head_prenorm(q1, k1, q2, k2, v, -lam, causal, mode="diff")
+        assert np.allclose(O, O_neg, atol=1e-13)
+    S1, S2 = q1 @ k1.T / 2.0, q2 @ k2.T / 2.0
+    assert np.allclose(ref.map_weights(S1, S2, lam, "sum").sum(axis=1), 1.0 + lam, atol=1e-13)
+    try:
+        ref.map_weights(S1, S2, lam, "difference")
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("an unknown mode was accepted")
+
+
 PINS = [pin_worked_example, pin_large_scores, pin_row_sums, pin_lambda_zero_is_attention, pin_map2_alone,
         pin_equal_maps, pin_causal_row0, pin_rmsnorm_hand, pin_lambda_hand, pin_brute_force,
-        pin_decode_is_last_prefill_row, pin_sampled_rows]
+        pin_decode_is_last_prefill_row, pin_sampled_rows, pin_mode_lambda_zero, pin_mode_sum]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -297,8 +346,20 @@ def _mut_lambda_sign(lq1, lk1, lq2, lk2, lambda_init):
     return float(np.exp(np.dot(lq1, lk1)) + np.exp(np.dot(lq2, lk2)) + lambda_init)
 
 
-def _mut_head_swap(q1, k1, q2, k2, v, lam, causal, rows=None):
-    return _orig_head(q1, k2, q2, k1, v, lam, causal, rows)
+def _mut_head_swap(q1, k1, q2, k2, v, lam, causal, rows=None, mode="diff"):
+    return _orig_head(q1, k2, q2, k1, v, lam, causal, rows, mode)
+
+
+def _mut_sum_subtracts(S1, S2, lam, mode="diff"):
+    if mode == "lambda_zero":
+        return ref.softmax_rows(S1)
+    return ref.softmax_rows(S1) - float(lam) * ref.softmax_rows(S2)
+
+
+def _mut_zero_keeps_map2(S1, S2, lam, mode="diff"):
+    if mode == "sum":
+        return ref.softmax_rows(S1) + float(lam) * ref.softmax_rows(S2)
+    return ref.softmax_rows(S1) - float(lam) * ref.softmax_rows(S2)
 
 
 def _mut_decode_maps(q1, q2, k1, k2, v, lam):
@@ -321,6 +382,8 @@ MUTANTS = {
     "lambda_reparam_sign": ("lambda_reparam", _mut_lambda_sign),
     "keys_of_maps_swapped": ("diffattn_head_prenorm", _mut_head_swap),
     "decode_map2_uses_k1": ("decode_head_prenorm", _mut_decode_maps),
+    "sum_mode_subtracts": ("map_weights", _mut_sum_subtracts),
+    "lambda_zero_keeps_map2": ("map_weights", _mut_zero_keeps_map2),
 }
 
 

@@ -19,6 +19,8 @@ SIGNATURES = {
     "diffattn_lambda": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_float, _vp, _vp]),
     "diffattn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                               _vp, _c_float, _vp, _c_float, _vp]),
+    "diffattn_fwd_mode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _vp, _c_float, _vp, _c_float, _c_int, _vp]),
     "diffattn_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _c_float,
                                  _vp, _c_float, _vp, _c_size, _vp]),

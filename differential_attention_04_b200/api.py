@@ -14,6 +14,8 @@ from ._lib import lib
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
 F32, BF16 = 0, 1
+# how the two maps are combined: softmax(S1) + c softmax(S2), c = -lambda, 0, +lambda
+MODE_DIFF, MODE_LAMBDA_ZERO, MODE_SUM = 0, 1, 2
 
 
 class DiffAttnError(RuntimeError):
@@ -60,8 +62,11 @@ def diffattn_lambda(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor, lk2
 
 def diffattn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor, lambda_init: float,
                  rms_w: torch.Tensor, eps: float = 1e-5, causal: bool = True,
-                 out: torch.Tensor | None = None) -> torch.Tensor:
-    """Prefill.  q, k: [B, N, H, 2, d]; v: [B, N, H, 2d]; lam: device fp32 scalar; rms_w: fp32 [2d]."""
+                 out: torch.Tensor | None = None, mode: int = MODE_DIFF) -> torch.Tensor:
+    """Prefill.  q, k: [B, N, H, 2, d]; v: [B, N, H, 2d]; lam: device fp32 scalar; rms_w: fp32 [2d].
+
+    ``mode`` (MODE_DIFF, MODE_LAMBDA_ZERO, MODE_SUM) picks the combination of
+    the two maps; MODE_DIFF is the differential attention itself."""
     _dev(q, k, v, lam, rms_w)
     B, N, H, two, d = q.shape
     if two != 2 or k.shape != q.shape or tuple(v.shape) != (B, N, H, 2 * d):
@@ -76,9 +81,14 @@ def diffattn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.T
         raise ValueError("q, k, v must share one dtype")
     if out is None:
         out = torch.empty_like(v)
-    _check("diffattn_fwd", lib().diffattn_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)), _ptr(lam),
-        float(lambda_init), _ptr(rms_w), float(eps), _stream()))
+    if mode == MODE_DIFF:
+        _check("diffattn_fwd", lib().diffattn_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)), _ptr(lam),
+            float(lambda_init), _ptr(rms_w), float(eps), _stream()))
+    else:
+        _check("diffattn_fwd_mode", lib().diffattn_fwd_mode(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)), _ptr(lam),
+            float(lambda_init), _ptr(rms_w), float(eps), int(mode), _stream()))
     return out
 
 

@@ -124,7 +124,16 @@ int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const 
 int diffattn_fwd(const void* q, const void* k, const void* v, void* o, int dtype, int B, int N, int H, int d,
                  int causal, const float* lambda, float lambda_init, const float* rms_w, float eps,
                  cudaStream_t stream) {
+  return diffattn_fwd_mode(q, k, v, o, dtype, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
+                           DIFFATTN_MODE_DIFF, stream);
+}
+
+int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o, int dtype, int B, int N, int H,
+                      int d, int causal, const float* lambda, float lambda_init, const float* rms_w, float eps,
+                      int mode, cudaStream_t stream) {
   if (B < 1 || H < 1 || N < 0 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
   if (dtype != DIFFATTN_F32 && dtype != DIFFATTN_BF16) return DIFFATTN_ERR_INVALID_ARG;
   if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
   if (N == 0) return DIFFATTN_OK;
@@ -135,7 +144,7 @@ int diffattn_fwd(const void* q, const void* k, const void* v, void* o, int dtype
     if (d > 128) return DIFFATTN_ERR_UNSUPPORTED;
     return cuda_status(launch_prefill_simt_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                                static_cast<const float*>(v), static_cast<float*>(o), B, N, H, d,
-                                               causal, lambda, lambda_init, rms_w, eps, stream));
+                                               causal, lambda, lambda_init, rms_w, eps, mode, stream));
   }
   if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv, to;
@@ -147,7 +156,8 @@ int diffattn_fwd(const void* q, const void* k, const void* v, void* o, int dtype
   if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
   return cuda_status(
-      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, ctl, stream));
+      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, ctl,
+                           stream));
 }
 
 size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen) {

@@ -19,15 +19,20 @@ cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, 
 // CUDA-core prefill for float32 tensors, any 1 <= d <= 128.
 cudaError_t launch_prefill_simt_f32(const float* q, const float* k, const float* v, float* o, int B, int N, int H,
                                     int d, int causal, const float* lambda, float lambda_init, const float* rms_w,
-                                    float eps, cudaStream_t stream);
+                                    float eps, int mode, cudaStream_t stream);
+
+// Coefficient c of map 2 in D = softmax(S1) + c softmax(S2) for a diffattn_mode.
+__host__ __device__ inline float map2_coefficient(int mode, float lam) {
+  return mode == 0 ? -lam : (mode == 2 ? lam : 0.0f);
+}
 
 // Tensor-core (tcgen05) prefill for bf16 tensors, d in {64, 128}.  tq/tk map
-// [B, N, H*2, d]; tv maps [B, N, H, 2d]; boxes are 64 columns x 128 rows with
-// 128-byte swizzle.
+// [B, N, H*2, d]; tv and to map [B, N, H, 2d]; boxes are 64 columns x 128
+// rows with 128-byte swizzle.
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
-                                 const float* rms_w, float eps, DevCtl ctl, cudaStream_t stream);
+                                 const float* rms_w, float eps, int mode, DevCtl ctl, cudaStream_t stream);
 
 // Split-KV decode (bf16, d = 128).
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);

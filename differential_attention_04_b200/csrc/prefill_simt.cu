@@ -28,7 +28,7 @@ constexpr int kMaxU = 8;  // ceil(2 * 128 / 32)
 __global__ void __launch_bounds__(256) prefill_simt_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, float* __restrict__ o,
     int N, int H, int d, int causal, const float* __restrict__ lambda_ptr, float lambda_init,
-    const float* __restrict__ rms_w, float eps) {
+    const float* __restrict__ rms_w, float eps, int mode) {
   extern __shared__ float smem[];
   const int kstride = (d % 2 == 0) ? d + 1 : d;  // odd row pitch: conflict-free column reads
   const int dv = 2 * d;
@@ -142,19 +142,19 @@ __global__ void __launch_bounds__(256) prefill_simt_f32_kernel(
     }
   }
 
-  const float lam = *lambda_ptr;
+  const float coef2 = map2_coefficient(mode, *lambda_ptr);  // c in softmax(S1) + c softmax(S2)
   const float out_scale = 1.0f - lambda_init;
 #pragma unroll
   for (int rr = 0; rr < kRowsPerWarp; ++rr) {
     const int qi = q0 + warp * kRowsPerWarp + rr;
     if (qi >= N) continue;
-    const float inv1 = 1.0f / l1[rr], inv2 = lam / l2[rr];
+    const float inv1 = 1.0f / l1[rr], inv2 = coef2 / l2[rr];
     float ov[kMaxU];
     float ss = 0.f;
 #pragma unroll
     for (int u = 0; u < kMaxU; ++u) {
       const int c = lane + 32 * u;
-      ov[u] = (c < dv) ? o1[rr][u] * inv1 - o2[rr][u] * inv2 : 0.f;
+      ov[u] = (c < dv) ? o1[rr][u] * inv1 + o2[rr][u] * inv2 : 0.f;
       ss = fmaf(ov[u], ov[u], ss);
     }
 #pragma unroll
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(256) prefill_simt_f32_kernel(
 
 cudaError_t launch_prefill_simt_f32(const float* q, const float* k, const float* v, float* o, int B, int N, int H,
                                     int d, int causal, const float* lambda, float lambda_init, const float* rms_w,
-                                    float eps, cudaStream_t stream) {
+                                    float eps, int mode, cudaStream_t stream) {
   const int kstride = (d % 2 == 0) ? d + 1 : d;
   const size_t smem =
       sizeof(float) * (2 * kRowsPerCta * d + 2 * kKeysPerTile * kstride + kKeysPerTile * 2 * d);
@@ -179,7 +179,7 @@ cudaError_t launch_prefill_simt_f32(const float* q, const float* k, const float*
   if (e != cudaSuccess) return e;
   dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, H, B);
   prefill_simt_f32_kernel<<<grid, 256, smem, stream>>>(q, k, v, o, N, H, d, causal, lambda, lambda_init, rms_w,
-                                                       eps);
+                                                       eps, mode);
   return cudaGetLastError();
 }
 

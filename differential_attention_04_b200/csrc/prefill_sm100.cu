@@ -106,6 +106,7 @@ struct PrefillParams {
   __nv_bfloat16* o;
   int N, H, causal, n_qtiles;
   const float* lambda;
+  int mode;  // diffattn_mode: how map 2 enters the combination
   float lambda_init;
   const float* rms_w;
   float eps;
@@ -409,13 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int HALF = C::HALF;
   constexpr int NC = HALF / 4;  // float4 chunks per exchanged row
   cluster_sync_all();  // both CTAs: main loops drained, buffers free
-  const float lam = *p.lambda;
+  const float coef2 = map2_coefficient(p.mode, *p.lambda);  // c in softmax(S1) + c softmax(S2)
   const int own0 = (rank == 0) ? 0 : HALF;   // columns this CTA finishes
   const int send0 = (rank == 0) ? HALF : 0;  // columns it hands to the partner
   float y[HALF];
   float ss = 0.f;
   if (is_sm) {
-    const float inv = (rank == 0) ? 1.0f / l_run : -lam / l_run;
+    const float inv = (rank == 0) ? 1.0f / l_run : coef2 / l_run;
     float* srow = stage + r * HALF;
 #pragma unroll
     for (int c = 0; c < HALF / 32; ++c) {
@@ -520,7 +521,7 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
-                                 const float* rms_w, float eps, DevCtl ctl, cudaStream_t stream) {
+                                 const float* rms_w, float eps, int mode, DevCtl ctl, cudaStream_t stream) {
   PrefillParams prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.N = N;
@@ -528,6 +529,7 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.causal = causal ? 1 : 0;
   prm.n_qtiles = (N + kBM - 1) / kBM;
   prm.lambda = lambda;
+  prm.mode = mode;
   prm.lambda_init = lambda_init;
   prm.rms_w = rms_w;
   prm.eps = eps;

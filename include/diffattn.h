@@ -97,6 +97,31 @@ int diffattn_fwd(const void* q, const void* k, const void* v, void* o,
                  const float* lambda, float lambda_init, const float* rms_w,
                  float eps, cudaStream_t stream);
 
+/* How the two maps are combined (peer review "Differential Transformer",
+ * Weaknesses, second bullet, and Questions, first bullet: the controls it
+ * asks for).  D = softmax(S1) + c * softmax(S2), then O = D V:
+ *   DIFFATTN_MODE_DIFF        c = -lambda  (the method; diffattn_fwd)
+ *   DIFFATTN_MODE_LAMBDA_ZERO c = 0        (lambda fixed to 0: one softmax map,
+ *                                           same widths, norm and scale)
+ *   DIFFATTN_MODE_SUM         c = +lambda  (the two maps added)          */
+typedef enum {
+  DIFFATTN_MODE_DIFF = 0,
+  DIFFATTN_MODE_LAMBDA_ZERO = 1,
+  DIFFATTN_MODE_SUM = 2
+} diffattn_mode;
+
+/*
+ * diffattn_fwd_mode -- diffattn_fwd with the combination of the two maps
+ * chosen by `mode` (a diffattn_mode).  All other arguments, layouts and
+ * errors are those of diffattn_fwd; an unknown mode gives
+ * DIFFATTN_ERR_INVALID_ARG.  In DIFFATTN_MODE_LAMBDA_ZERO the lambda pointer
+ * must still be valid (it is read, then multiplied by zero).
+ */
+int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o,
+                      int dtype, int B, int N, int H, int d, int causal,
+                      const float* lambda, float lambda_init, const float* rms_w,
+                      float eps, int mode, cudaStream_t stream);
+
 /*
  * diffattn_decode_workspace_size -- bytes of device workspace that
  * diffattn_decode needs for S sequences of at most max_seqlen cached keys.

@@ -65,6 +65,13 @@ def test_validation_without_gpu(L):
     assert args(fake, api.F32, 1, 16, 2, 129) == api.ERR_UNSUPPORTED
     assert args(fake, api.BF16, 1 << 16, 1 << 16, 2, 128) == api.ERR_INVALID_ARG  # > 2^31 elements
     assert args(nul, api.BF16, 1, 0, 2, 128) == api.OK  # N = 0 is a no-op
+    # prefill with a combination mode: unknown modes are rejected
+    margs = lambda q, mode: L.diffattn_fwd_mode(q, q, q, q, api.BF16, 1, 16, 2, 128, 1, q, 0.5, q, 1e-5, mode, nul)
+    for bad in (-1, 3, 7):
+        assert margs(fake, bad) == api.ERR_INVALID_ARG
+    assert margs(nul, api.MODE_SUM) == api.ERR_INVALID_ARG
+    assert L.diffattn_fwd_mode(nul, nul, nul, nul, api.BF16, 1, 0, 2, 128, 1, nul, 0.5, nul, 1e-5,
+                               api.MODE_LAMBDA_ZERO, nul) == api.OK
     # decode
     dec = lambda q, d, ws, wsb, S=4: L.diffattn_decode(q, q, q, q, 100, q, S, 2, d, q, 0.5, q, 1e-5, ws, wsb, nul)
     assert dec(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG

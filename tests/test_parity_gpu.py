@@ -177,6 +177,51 @@ def test_bf16_score_jumps():
     assert_close(wl.to_f64(y), oracle_prefill(inp))
 
 
+MODE_NAMES = {api.MODE_LAMBDA_ZERO: "lambda_zero", api.MODE_SUM: "sum"}
+
+
+def _oracle_mode(inp, mode):
+    f = wl.to_f64
+    return ref.diffattn_fwd(f(inp.q), f(inp.k), f(inp.v), oracle_lambda(inp), inp.lambda_init, f(inp.rms_w),
+                            inp.eps, inp.causal, mode=MODE_NAMES[mode])
+
+
+@pytest.mark.parametrize("mode", sorted(MODE_NAMES))
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_control_modes(mode, d, causal):
+    # the review's controls: lambda fixed to 0 (one map) and the maps added
+    inp = wl.make_prefill(1, 200, 2, d, causal=causal, dtype="bf16", lambda_init=0.5, w="normal", seed=31 + d,
+                          device="cuda")
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+    y = api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, causal, mode=mode)
+    torch.cuda.synchronize()
+    assert_close(wl.to_f64(y), _oracle_mode(inp, mode))
+
+
+@pytest.mark.parametrize("mode", sorted(MODE_NAMES))
+def test_fp32_control_modes(mode):
+    inp = wl.make_prefill(2, 70, 3, 32, causal=True, dtype="f32", lambda_init=0.3, w="normal", seed=41,
+                          device="cuda")
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+    y = api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, True, mode=mode)
+    torch.cuda.synchronize()
+    assert_close(wl.to_f64(y), _oracle_mode(inp, mode), fp32=True)
+
+
+def test_lambda_zero_ignores_map2():
+    inp = wl.make_prefill(1, 300, 2, 128, causal=True, dtype="bf16", seed=43, device="cuda")
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+    y1 = api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, True,
+                          mode=api.MODE_LAMBDA_ZERO)
+    inp.q[:, :, :, 1].normal_()
+    inp.k[:, :, :, 1].mul_(3.0)
+    y2 = api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, True,
+                          mode=api.MODE_LAMBDA_ZERO)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
 def test_output_only_written_in_bounds():
     inp = wl.make_prefill(1, 200, 2, 128, causal=True, dtype="bf16", seed=3, device="cuda")
     lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)

@@ -20,6 +20,7 @@ step), and the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -41,8 +42,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=20)
+    # defaults: about 1 s of timed, back-to-back steps (a sustained loop, so the
+    # clocks seen are those under the power cap), after 0.1 s of warm-up
+    ap.add_argument("--steps", type=int, default=1600)
+    ap.add_argument("--warmup", type=int, default=150)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
@@ -120,12 +123,20 @@ class ClockSampler:
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,timestamp")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t_begin = self.t_end = None
+
+    def mark_begin(self):
+        """Host time at the start of the timed region (samples before it are dropped)."""
+        self.t_begin = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
 
     def start(self):
         try:
@@ -152,9 +163,20 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
+            if len(parts) >= 10:
                 rows.append(parts)
         os.unlink(self.path)
+        # keep the samples taken inside the timed region (nvidia-smi stamps each
+        # line with the host's local time)
+        if self.t_begin is not None and self.t_end is not None:
+            def stamp(r):
+                try:
+                    return datetime.datetime.strptime(r[9], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    return None
+            inside = [r for r in rows if stamp(r) is not None and self.t_begin <= stamp(r) <= self.t_end]
+            if inside:
+                rows = inside
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -166,6 +188,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(pw) if pw else None,
+                "power_w_median": statistics.median(pw) if pw else None,
                 "reasons": reasons, "samples": len(rows)}
 
 
@@ -314,6 +337,7 @@ def run_ours(args):
     clocks.start()
     barrier()
     torch.cuda.synchronize()
+    clocks.mark_begin()
     t0.record()
     for i in range(K):
         api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init, out=lam)
@@ -322,6 +346,7 @@ def run_ours(args):
         ev[i][1].record()
     t1.record()
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier()
     clk = clocks.stop()
     ms_total = reduce_max(t0.elapsed_time(t1))
@@ -336,6 +361,14 @@ def run_ours(args):
     value = job_throughput(flops_metric, world, ms_step) / 1e12
     achieved = flops_alg / (kern_ms * 1e-3) / 1e12
     traffic = read_profile_traffic("prefill_sm100_prefill_3b")
+    # The kernel is timed inside a loop of back-to-back steps: for a loop of a
+    # second or more the matching denominator is the sustained GEMM figure
+    # (measured as a seconds-long loop under the same power cap); shorter runs
+    # use the burst figure.
+    sustained = ms_total >= 1000.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    peak_kind = (f"sustained (timed loop {ms_total / 1e3:.2f} s)" if sustained
+                 else f"burst (timed loop {ms_total / 1e3:.2f} s < 1 s)")
 
     # end to end through the public API: pinned host inputs, H2D inside the timed region, D2H of the output
     E = max(1, args.e2e_steps)
@@ -379,10 +412,11 @@ def run_ours(args):
             "l2": f"inputs larger than L2: q+k+v = {3 * inp.q.numel() * 2 / 1e6:.0f} MB per step > 126 MB",
             "parallelism": f"replicas x{world} (one process per GPU, no collective on the path)",
         },
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
                      "kernel": "prefill_sm100_kernel<128>", "kernel_ms": kern_ms,
-                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "peak_source": f"{peak_src} bf16 dense, {peak_kind}",
+                     "frac_of_burst": achieved / peaks["bf16_tflops"],
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},

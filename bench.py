@@ -49,6 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-qk8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
@@ -243,6 +244,55 @@ def cpu_baseline(inp, budget_s):
 
 # --------------------------------------------------------------- reference --
 
+def bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K):
+    """The e4m3 query/key variant on the same workload: a step quantises q and k
+    (one absmax scale per batch, head and map) and runs the prefill whose
+    scores are 8-bit tensor-core products."""
+    import torch
+
+    B, N, H, _, d = inp.q.shape
+    qc, qs = api.quantize_qk(inp.q)
+    kc, ks = api.quantize_qk(inp.k)
+
+    def quant():
+        api.quantize_qk(inp.q, qc, qs)
+        api.quantize_qk(inp.k, kc, ks)
+
+    def fwd():
+        api.diffattn_fwd_qk8(qc, qs, kc, ks, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
+
+    for _ in range(5):
+        quant()
+        fwd()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for e0, e1, e2 in ev:
+        e0.record()
+        quant()
+        e1.record()
+        fwd()
+        e2.record()
+    torch.cuda.synchronize()
+    q_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b, _ in ev))
+    f_ms = reduce_max(statistics.mean(b.elapsed_time(c) for _, b, c in ev))
+    flops_metric = prefill_flops(B, N, H, d, inp.causal, "metric")
+    flops_alg = prefill_flops(B, N, H, d, inp.causal, "algorithmic")
+    # a third of the algorithmic flops (the scores, 4d of 12d per pair) run on the
+    # 8-bit path at twice the bf16 rate: the mixed peak is 1 / (1/6 + 2/3) = 1.2 x bf16
+    bf16_peak = peaks["bf16_tflops"]
+    mixed = 1.2 * bf16_peak
+    achieved = flops_alg / (f_ms * 1e-3) / 1e12
+    return {"metric": "DiffAttn fwd TFLOP/s, e4m3 queries/keys (quantise + prefill)",
+            "value": flops_metric / ((q_ms + f_ms) * 1e-3) / 1e12, "unit": "TFLOP/s", "steps": K,
+            "ms_per_step": q_ms + f_ms, "quantize_ms": q_ms, "prefill_ms": f_ms,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": mixed, "unit": "TFLOP/s",
+                         "frac": achieved / mixed, "traffic": None, "kernel": "prefill_sm100_kernel<128, e4m3>",
+                         "peak_source": f"{peak_src} bf16 dense (burst) x 1.2: scores on the 8-bit path at the "
+                                        "nominal 2x rate"},
+            "gpu_launches": 7 * K}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -424,6 +474,8 @@ def run_ours(args):
         "clocks": clk,
     }
 
+    if not args.no_qk8 and d == 128:
+        line["qk8"] = bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8))
     if not args.no_decode:
         line["decode"] = bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world)
     del inp, y

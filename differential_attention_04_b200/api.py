@@ -92,6 +92,45 @@ def diffattn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.T
     return out
 
 
+def quantize_qk(x: torch.Tensor, codes: torch.Tensor | None = None,
+                scales: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """e4m3 codes (uint8, x's shape) and float32 scales [B, H, 2] of a bf16 q or k [B, N, H, 2, d]:
+    one absmax scale per (batch, head, map)."""
+    _dev(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 5 or x.shape[3] != 2:
+        raise ValueError("x must be bfloat16 [B, N, H, 2, d]")
+    B, N, H, _, d = x.shape
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, 2), dtype=torch.float32, device=x.device)
+    _dev(codes, scales)
+    if codes.shape != x.shape or codes.dtype != torch.uint8 or scales.numel() != B * H * 2 or \
+            scales.dtype != torch.float32:
+        raise ValueError("codes must be uint8 like x and scales float32 [B, H, 2]")
+    _check("diffattn_quantize_qk", lib().diffattn_quantize_qk(_ptr(x), B, N, H, d, _ptr(codes), _ptr(scales),
+                                                              _stream()))
+    return codes, scales
+
+
+def diffattn_fwd_qk8(q_codes: torch.Tensor, q_scales: torch.Tensor, k_codes: torch.Tensor, k_scales: torch.Tensor,
+                     v: torch.Tensor, lam: torch.Tensor, lambda_init: float, rms_w: torch.Tensor, eps: float = 1e-5,
+                     causal: bool = True, out: torch.Tensor | None = None, mode: int = MODE_DIFF) -> torch.Tensor:
+    """Prefill with e4m3 queries and keys (as quantize_qk returns them); v, out: bf16 [B, N, H, 2d]."""
+    _dev(q_codes, q_scales, k_codes, k_scales, v, lam, rms_w)
+    B, N, H, two, d = q_codes.shape
+    if q_codes.dtype != torch.uint8 or k_codes.dtype != torch.uint8 or k_codes.shape != q_codes.shape or two != 2:
+        raise ValueError("q_codes, k_codes must be uint8 [B, N, H, 2, d]")
+    if v.dtype != torch.bfloat16 or tuple(v.shape) != (B, N, H, 2 * d):
+        raise ValueError("v must be bfloat16 [B, N, H, 2d]")
+    if out is None:
+        out = torch.empty_like(v)
+    _check("diffattn_fwd_qk8", lib().diffattn_fwd_qk8(
+        _ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v), _ptr(out), B, N, H, d,
+        int(bool(causal)), _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode), _stream()))
+    return out
+
+
 def decode_workspace_size(S: int, H: int, d: int, max_seqlen: int) -> int:
     return int(lib().diffattn_decode_workspace_size(S, H, d, max_seqlen))
 

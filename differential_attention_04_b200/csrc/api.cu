@@ -60,16 +60,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4-D bf16 map over a row-major tensor with dims (innermost first) d0..d3,
-// box = 64 x 1 x 128 x 1 elements, 128-byte swizzle, zero fill out of bounds.
-bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+// 4-D map over a row-major tensor with dims (innermost first) d0..d3 of bf16
+// (esize 2) or byte (esize 1) elements; box = 128 bytes x 1 x 128 x 1,
+// 128-byte swizzle, zero fill out of bounds.
+bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+               int esize = 2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const uint64_t e = static_cast<uint64_t>(esize);
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint64_t strides[3] = {d0 * e, d0 * d1 * e, d0 * d1 * d2 * e};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+            const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -156,8 +160,43 @@ int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o, int 
   if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
   return cuda_status(
-      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, ctl,
-                           stream));
+      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, nullptr,
+                           nullptr, ctl, stream));
+}
+
+int diffattn_quantize_qk(const void* x, int B, int N, int H, int d, void* codes, float* scales,
+                         cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 1 || d < 8 || d % 8 != 0) return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!x || !codes || !scales) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return DIFFATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * 2 > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  return cuda_status(launch_quantize_qk(x, B, N, H, d, codes, scales, stream));
+}
+
+int diffattn_fwd_qk8(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,
+                     const void* v, void* o, int B, int N, int H, int d, int causal, const float* lambda,
+                     float lambda_init, const float* rms_w, float eps, int mode, cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 0 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (N == 0) return DIFFATTN_OK;
+  if (!q_codes || !q_scales || !k_codes || !k_scales || !v || !o || !lambda || !rms_w)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !aligned16(v) || !aligned16(o)) return DIFFATTN_ERR_INVALID_ARG;
+  if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_4d(&tq, q_codes, d, 2ull * H, N, B, 1) || !encode_4d(&tk, k_codes, d, 2ull * H, N, B, 1) ||
+      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
+    return DIFFATTN_ERR_CUDA;
+  DevCtl ctl;
+  cudaError_t e = status_ptr(&ctl.status);
+  if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  ctl.limit_ns = g_wait_limit_ns.load();
+  return cuda_status(launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
+                                          mode, q_scales, k_scales, ctl, stream));
 }
 
 size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen) {

@@ -128,6 +128,17 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (8-bit float inputs, fp32 accumulate).
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16; A is read from tensor memory.
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {
@@ -252,6 +263,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          | (1u << 10)                             // B format: bf16
          | ((a_mn ? 1u : 0u) << 15)               // A major
          | ((b_mn ? 1u : 0u) << 16)               // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N >> 3
+         | (static_cast<uint32_t>(M >> 4) << 24); // M >> 4
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A/B (both K-major) and
+// fp32 D; K = 32 per instruction.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                // D format: f32
+         | (0u << 7)                              // A format: e4m3
+         | (0u << 10)                             // B format: e4m3
          | (static_cast<uint32_t>(N >> 3) << 17)  // N >> 3
          | (static_cast<uint32_t>(M >> 4) << 24); // M >> 4
 }

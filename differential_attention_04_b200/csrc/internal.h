@@ -26,13 +26,20 @@ __host__ __device__ inline float map2_coefficient(int mode, float lam) {
   return mode == 0 ? -lam : (mode == 2 ? lam : 0.0f);
 }
 
-// Tensor-core (tcgen05) prefill for bf16 tensors, d in {64, 128}.  tq/tk map
-// [B, N, H*2, d]; tv and to map [B, N, H, 2d]; boxes are 64 columns x 128
-// rows with 128-byte swizzle.
+// Tensor-core (tcgen05) prefill, d in {64, 128} for bf16 queries and keys,
+// d = 128 for e4m3 ones (q_scale, k_scale non-null).  tq/tk map
+// [B, N, H*2, d]; tv and to map [B, N, H, 2d]; boxes are 128 bytes x 128 rows
+// with 128-byte swizzle.
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
-                                 const float* rms_w, float eps, int mode, DevCtl ctl, cudaStream_t stream);
+                                 const float* rms_w, float eps, int mode, const float* q_scale,
+                                 const float* k_scale, DevCtl ctl, cudaStream_t stream);
+
+// e4m3 codes of a bf16 [B, N, H, 2, d] tensor with one float32 scale per
+// (batch, head, map) (scales: [B][H][2], also the absmax accumulator).
+cudaError_t launch_quantize_qk(const void* x, int B, int N, int H, int d, void* codes, float* scales,
+                               cudaStream_t stream);
 
 // Split-KV decode (bf16, d = 128).
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);

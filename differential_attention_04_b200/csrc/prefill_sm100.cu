@@ -62,15 +62,21 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kOverflowGuard = 64.0f;    // log2 units
 
-template <int D>
+// QK8: queries and keys arrive as e4m3 codes (one byte each) with a float32
+// scale per (batch, head, map); S is then a kind::f8f6f4 product.  Otherwise
+// they are bf16 and S is a kind::f16 product.
+template <int D, bool QK8>
 struct Cfg {
   static constexpr int DV = 2 * D;
   static constexpr int HALF = D;                 // output columns owned by each CTA
-  static constexpr int QBLK = D / 64;            // 64-column swizzle blocks per Q/K row
+  static constexpr int QE = QK8 ? 1 : 2;         // bytes per Q/K element
+  static constexpr int QBOX = 128 / QE;          // Q/K elements per 128-byte swizzle row
+  static constexpr int QBLK = D / QBOX;          // 128-byte swizzle blocks per Q/K row
+  static constexpr int KSTEP = QK8 ? 32 : 16;    // K of one S instruction
   static constexpr int VBLK = DV / 64;           // 64-column blocks per V row
-  static constexpr int BLK_BYTES = 128 * 128;    // one [128 rows][64 bf16] block
-  static constexpr int Q_BYTES = kBM * D * 2;
-  static constexpr int K_BYTES = kBN * D * 2;
+  static constexpr int BLK_BYTES = 128 * 128;    // one [128 rows][128 bytes] block
+  static constexpr int Q_BYTES = kBM * D * QE;
+  static constexpr int K_BYTES = kBN * D * QE;
   static constexpr int V_BYTES = kBN * DV * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
@@ -106,6 +112,8 @@ struct PrefillParams {
   __nv_bfloat16* o;
   int N, H, causal, n_qtiles;
   const float* lambda;
+  const float* q_scale;  // QK8 only: float32 [B][H][2], one scale per (batch, head, map)
+  const float* k_scale;
   int mode;  // diffattn_mode: how map 2 enters the combination
   float lambda_init;
   const float* rms_w;
@@ -123,12 +131,12 @@ __device__ __forceinline__ void tmem_ld_wait4(uint32_t (&a)[32], uint32_t (&b)[3
   tmem_ld_wait(d);
 }
 
-template <int D>
+template <int D, bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                          const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
                          const PrefillParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, QK8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -189,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
 #pragma unroll
       for (int blk = 0; blk < C::QBLK; ++blk)
-        tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * 64, c1, qtile * kBM, b);
+        tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * C::QBOX, c1, qtile * kBM, b);
       int issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j & 1;
@@ -198,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
 #pragma unroll
         for (int blk = 0; blk < C::QBLK; ++blk)
-          tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * 64, c1, j * kBN, b);
+          tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * C::QBOX, c1,
+                      j * kBN, b);
         issued = j + 1;
       }
       // make sure nothing is still landing in shared memory before the epilogue reuses it
@@ -226,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_s = QK8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       // O += P_t V_t, with P from buffer t % 2 and V from stage t % 2
@@ -254,12 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(&bars->k_full[st], (j >> 1) & 1, wc))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / C::KSTEP; ++kk) {  // each instruction takes 32 bytes of every row
           const int blk = kk >> 2;
           const uint32_t koff = (kk & 3) * 32;
           const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + koff, 16, 1024);
-          umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          if constexpr (QK8)
+            umma_ss_f8(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->k_empty[st]);
         umma_commit(&bars->s_full);
@@ -282,7 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float m_run = -INFINITY, l_run = 0.f;
   bool sm_ok = true;
   if (is_sm) {
-    const float sc = kLog2e * rsqrtf(static_cast<float>(D));
+    float sc = kLog2e * rsqrtf(static_cast<float>(D));
+    if constexpr (QK8) {  // scores of the codes times the two groups' scales
+      const int g = (b * p.H + h) * 2 + static_cast<int>(rank);
+      sc *= __ldg(p.q_scale + g) * __ldg(p.k_scale + g);
+    }
     // O and l *= alpha (the whole warp takes part; alpha = 1 leaves a row as it is)
     auto rescale_o = [&](float alpha) {
 #pragma unroll
@@ -496,11 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool QK8>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const PrefillParams& prm, int B, cudaStream_t stream) {
-  using C = Cfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  using C = Cfg<D, QK8>;
+  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -515,13 +531,14 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D>, tq, tk, tv, to, prm);
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8>, tq, tk, tv, to, prm);
 }
 
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
-                                 const float* rms_w, float eps, int mode, DevCtl ctl, cudaStream_t stream) {
+                                 const float* rms_w, float eps, int mode, const float* q_scale,
+                                 const float* k_scale, DevCtl ctl, cudaStream_t stream) {
   PrefillParams prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.N = N;
@@ -529,14 +546,18 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.causal = causal ? 1 : 0;
   prm.n_qtiles = (N + kBM - 1) / kBM;
   prm.lambda = lambda;
+  prm.q_scale = q_scale;
+  prm.k_scale = k_scale;
   prm.mode = mode;
   prm.lambda_init = lambda_init;
   prm.rms_w = rms_w;
   prm.eps = eps;
   prm.status = ctl.status;
   prm.limit_ns = ctl.limit_ns;
-  if (d == 128) return launch_d<128>(tq, tk, tv, to, prm, B, stream);
-  if (d == 64) return launch_d<64>(tq, tk, tv, to, prm, B, stream);
+  const bool qk8 = q_scale != nullptr;
+  if (qk8) return d == 128 ? launch_d<128, true>(tq, tk, tv, to, prm, B, stream) : cudaErrorInvalidValue;
+  if (d == 128) return launch_d<128, false>(tq, tk, tv, to, prm, B, stream);
+  if (d == 64) return launch_d<64, false>(tq, tk, tv, to, prm, B, stream);
   return cudaErrorInvalidValue;
 }
 

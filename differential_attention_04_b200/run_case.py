@@ -1,6 +1,8 @@
 """Run one prefill or decode case a few times (e.g. under a profiler).
 
   python -m differential_attention_04_b200.run_case prefill --B 2 --N 4096 --H 12 --d 128 --causal 1 --iters 3
+  python -m differential_attention_04_b200.run_case prefill --qk8 1 ...   (e4m3 queries/keys: quantise + forward;
+                                                                          2: forward only; 3: quantise only)
   python -m differential_attention_04_b200.run_case decode --S 64 --H 12 --lmin 1024 --lmax 4096 --iters 3
 
 Inputs come from the seeded generators in ``workloads``; the output is not
@@ -26,6 +28,7 @@ def main(argv=None):
     ap.add_argument("--d", type=int, default=128)
     ap.add_argument("--causal", type=int, default=1)
     ap.add_argument("--dtype", default="bf16")
+    ap.add_argument("--qk8", type=int, default=0)
     ap.add_argument("--S", type=int, default=64)
     ap.add_argument("--lmin", type=int, default=1024)
     ap.add_argument("--lmax", type=int, default=4096)
@@ -39,8 +42,20 @@ def main(argv=None):
         inp = wl.make_prefill(a.B, a.N, a.H, a.d, causal=bool(a.causal), dtype=a.dtype, seed=a.seed, device=dev)
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
         y = torch.empty_like(inp.v)
-        run = lambda: api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
-                                       out=y)
+        if a.qk8:
+            qc, qs = api.quantize_qk(inp.q)
+            kc, ks = api.quantize_qk(inp.k)
+
+            def run():  # --qk8 1: quantise and forward; 2: forward only; 3: quantise only
+                if a.qk8 != 2:
+                    api.quantize_qk(inp.q, qc, qs)
+                    api.quantize_qk(inp.k, kc, ks)
+                if a.qk8 != 3:
+                    api.diffattn_fwd_qk8(qc, qs, kc, ks, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps,
+                                         inp.causal, out=y)
+        else:
+            run = lambda: api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps,
+                                           inp.causal, out=y)
     else:
         inp = wl.make_decode(a.S, a.H, a.d, a.lmin, a.lmax, seed=a.seed, device=dev)
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)

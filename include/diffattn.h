@@ -123,6 +123,44 @@ int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o,
                       float eps, int mode, cudaStream_t stream);
 
 /*
+ * Low-bit queries and keys (peer review "Differential Transformer",
+ * Strengths, the activation-outlier bullet, and Questions, the quantisation
+ * bullet: absmax quantisation per logit map and per head).
+ *
+ * diffattn_quantize_qk -- e4m3 codes of a bf16 query or key tensor, with one
+ * absmax scale per (batch, head, map):
+ *
+ *   scales[b][h][i] = max |x[b, :, h, i, :]| / 448   (float32; 1 if that max is 0)
+ *   codes[b, n, h, i, c] = e4m3(x[b, n, h, i, c] / scales[b][h][i])
+ *
+ * where e4m3 is the OCP FP8 E4M3 encoding, round to nearest even, saturating
+ * at +-448 (the largest finite value, where each group's absmax lands).
+ * x      : bf16 [B, N, H, 2, d] (the q or k of diffattn_fwd)
+ * codes  : device uint8 [B, N, H, 2, d], written
+ * scales : device float32 [B][H][2], written (also used as scratch)
+ * d must be a multiple of 8; B * H * 2 <= 65535.  Three stream-ordered
+ * kernels and one memset; no allocation.
+ * Errors: DIFFATTN_ERR_INVALID_ARG, DIFFATTN_ERR_UNSUPPORTED, DIFFATTN_ERR_CUDA.
+ */
+int diffattn_quantize_qk(const void* x, int B, int N, int H, int d, void* codes,
+                         float* scales, cudaStream_t stream);
+
+/*
+ * diffattn_fwd_qk8 -- the prefill of diffattn_fwd_mode with the scores taken
+ * from e4m3 queries and keys (codes and scales as diffattn_quantize_qk writes
+ * them): S_i = (Qcodes_i Kcodes_i^T) * q_scale * k_scale / sqrt(d), on the
+ * tensor cores' 8-bit path (fp32 accumulation).  P, V and the output stay
+ * bf16; everything after the scores is as in diffattn_fwd_mode.
+ * v, o : bf16 [B, N, H, 2d].  d must be 128 (DIFFATTN_ERR_UNSUPPORTED
+ * otherwise).  Other arguments and errors as in diffattn_fwd_mode.
+ */
+int diffattn_fwd_qk8(const void* q_codes, const float* q_scales,
+                     const void* k_codes, const float* k_scales,
+                     const void* v, void* o, int B, int N, int H, int d, int causal,
+                     const float* lambda, float lambda_init, const float* rms_w,
+                     float eps, int mode, cudaStream_t stream);
+
+/*
  * diffattn_decode_workspace_size -- bytes of device workspace that
  * diffattn_decode needs for S sequences of at most max_seqlen cached keys.
  * Returns 0 for invalid sizes.

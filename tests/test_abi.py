@@ -72,6 +72,17 @@ def test_validation_without_gpu(L):
     assert margs(nul, api.MODE_SUM) == api.ERR_INVALID_ARG
     assert L.diffattn_fwd_mode(nul, nul, nul, nul, api.BF16, 1, 0, 2, 128, 1, nul, 0.5, nul, 1e-5,
                                api.MODE_LAMBDA_ZERO, nul) == api.OK
+    # e4m3 queries/keys: quantiser and forward
+    qz = lambda x, N, d, B=1, H=2: L.diffattn_quantize_qk(x, B, N, H, d, x, x, nul)
+    assert qz(fake, 16, 12) == api.ERR_INVALID_ARG      # d not a multiple of 8
+    assert qz(fake, 0, 128) == api.ERR_INVALID_ARG
+    assert qz(nul, 16, 128) == api.ERR_INVALID_ARG
+    assert qz(fake, 16, 128, B=1 << 15, H=2) == api.ERR_UNSUPPORTED  # B*H*2 > 65535 groups
+    f8 = lambda x, N, d, mode=0: L.diffattn_fwd_qk8(x, x, x, x, x, x, 1, N, 2, d, 1, x, 0.5, x, 1e-5, mode, nul)
+    assert f8(fake, 16, 64) == api.ERR_UNSUPPORTED
+    assert f8(fake, 16, 128, mode=5) == api.ERR_INVALID_ARG
+    assert f8(nul, 16, 128) == api.ERR_INVALID_ARG
+    assert f8(nul, 0, 128) == api.OK
     # decode
     dec = lambda q, d, ws, wsb, S=4: L.diffattn_decode(q, q, q, q, 100, q, S, 2, d, q, 0.5, q, 1e-5, ws, wsb, nul)
     assert dec(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG

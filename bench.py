@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-qk8", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--bwd-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
@@ -243,6 +245,50 @@ def cpu_baseline(inp, budget_s):
 
 
 # --------------------------------------------------------------- reference --
+
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flops per FMA x 1965 MHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bench_bwd(api, inp, lam, reduce_max, barrier, K):
+    """The backward pass (training) on the same workload: dq, dk, dv, dlambda and
+    the norm weight's gradient for a seeded upstream gradient dy."""
+    import torch
+
+    B, N, H, _, d = inp.q.shape
+    g = torch.Generator(device=inp.q.device).manual_seed(4321)
+    dy = torch.randn(inp.v.shape, generator=g, device=inp.q.device).to(inp.v.dtype)
+    ws = torch.empty(api.bwd_workspace_size(B, N, H, d), dtype=torch.uint8, device=inp.q.device)
+
+    def step():
+        return api.diffattn_bwd(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
+                                workspace=ws)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev))
+    pairs = B * H * (N * (N + 1) // 2 if inp.causal else N * N)
+    # algorithmic: per visible (query, key) pair, 20 d flops -- recomputing both maps'
+    # scores (2 d MACs), dA = G V^T once (2 d), dV (2 d), dQ_i and dK_i (2 x 2 d)
+    alg = 20.0 * d * pairs
+    executed = 40.0 * d * pairs  # the row pass recomputes the forward; both gradient passes recompute S and dA
+    achieved = alg / (ms * 1e-3) / 1e12
+    return {"metric": "DiffAttn backward TFLOP/s (dq, dk, dv, dlambda, dw)", "value": achieved, "unit": "TFLOP/s",
+            "steps": K, "ms_per_step": ms, "flops_per_step_algorithmic": alg, "flops_per_step_executed": executed,
+            "roofline": {"bound": "alu", "achieved": executed / (ms * 1e-3) / 1e12, "peak": FP32_ALU_TFLOPS,
+                         "unit": "TFLOP/s", "frac": executed / (ms * 1e-3) / 1e12 / FP32_ALU_TFLOPS,
+                         "traffic": None, "kernel": "bwd_rows + bwd_keys + bwd_queries (CUDA cores, fp32)",
+                         "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz"},
+            "gpu_launches": 3 * K}
+
 
 def bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K):
     """The e4m3 query/key variant on the same workload: a step quantises q and k
@@ -474,6 +520,8 @@ def run_ours(args):
         "clocks": clk,
     }
 
+    if not args.no_bwd:
+        line["bwd"] = bench_bwd(api, inp, lam, reduce_max, barrier, args.bwd_steps)
     if not args.no_qk8 and d == 128:
         line["qk8"] = bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8))
     if not args.no_decode:

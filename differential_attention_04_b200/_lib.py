@@ -24,6 +24,10 @@ SIGNATURES = {
     "diffattn_quantize_qk": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "diffattn_fwd_qk8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                   _vp, _c_float, _vp, _c_float, _c_int, _vp]),
+    "diffattn_bwd_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "diffattn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
+                              _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "diffattn_lambda_bwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "diffattn_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _c_float,
                                  _vp, _c_float, _vp, _c_size, _vp]),

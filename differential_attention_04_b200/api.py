@@ -131,6 +131,45 @@ def diffattn_fwd_qk8(q_codes: torch.Tensor, q_scales: torch.Tensor, k_codes: tor
     return out
 
 
+def bwd_workspace_size(B: int, N: int, H: int, d: int) -> int:
+    return int(lib().diffattn_bwd_workspace_size(B, N, H, d))
+
+
+def diffattn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch.Tensor, lam: torch.Tensor,
+                 lambda_init: float, rms_w: torch.Tensor, eps: float = 1e-5, causal: bool = True,
+                 mode: int = MODE_DIFF, workspace: torch.Tensor | None = None):
+    """Backward of the prefill: (dq, dk, dv, dlambda, drms_w), float32, for the upstream gradient dy
+    (shaped like v).  q, k, v, dy share one dtype (bfloat16 or float32)."""
+    _dev(q, k, v, dy, lam, rms_w)
+    B, N, H, two, d = q.shape
+    if two != 2 or k.shape != q.shape or tuple(v.shape) != (B, N, H, 2 * d) or dy.shape != v.shape:
+        raise ValueError("shapes must be q, k: [B, N, H, 2, d] and v, dy: [B, N, H, 2d]")
+    dt = BF16 if q.dtype == torch.bfloat16 else F32 if q.dtype == torch.float32 else None
+    if dt is None or any(t.dtype != q.dtype for t in (k, v, dy)):
+        raise ValueError("q, k, v, dy must share one dtype, bfloat16 or float32")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dk, dv = torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)
+    dlam, dw = torch.empty(1, **f32), torch.empty(2 * d, **f32)
+    need = bwd_workspace_size(B, N, H, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("diffattn_bwd", lib().diffattn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dy), dt, B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+        _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream()))
+    return dq, dk, dv, dlam, dw
+
+
+def diffattn_lambda_bwd(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor, lk2: torch.Tensor,
+                        dlam: torch.Tensor):
+    """Gradients (dlq1, dlk1, dlq2, dlk2) of the lambda re-parameterisation for a device dlambda."""
+    _dev(lq1, lk1, lq2, lk2, dlam)
+    outs = [torch.empty_like(t) for t in (lq1, lk1, lq2, lk2)]
+    _check("diffattn_lambda_bwd", lib().diffattn_lambda_bwd(
+        _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), lq1.numel(), _ptr(dlam), *[_ptr(t) for t in outs], _stream()))
+    return tuple(outs)
+
+
 def decode_workspace_size(S: int, H: int, d: int, max_seqlen: int) -> int:
     return int(lib().diffattn_decode_workspace_size(S, H, d, max_seqlen))
 

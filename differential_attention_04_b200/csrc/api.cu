@@ -199,6 +199,38 @@ int diffattn_fwd_qk8(const void* q_codes, const float* q_scales, const void* k_c
                                           mode, q_scales, k_scales, ctl, stream));
 }
 
+size_t diffattn_bwd_workspace_size(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return 0;
+  return bwd_workspace_bytes(B, N, H, d);
+}
+
+int diffattn_bwd(const void* q, const void* k, const void* v, const void* dy, int dtype, int B, int N, int H, int d,
+                 int causal, const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                 float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace, size_t ws_bytes,
+                 cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (dtype != DIFFATTN_F32 && dtype != DIFFATTN_BF16) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !dy || !lambda || !rms_w || !dq || !dk || !dv || !dlambda || !drms_w)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (d > 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < bwd_workspace_bytes(B, N, H, d) || !aligned16(workspace))
+    return DIFFATTN_ERR_WORKSPACE;
+  return cuda_status(launch_bwd(q, k, v, dy, dtype == DIFFATTN_BF16, B, N, H, d, causal, lambda, lambda_init,
+                                rms_w, eps, mode, dq, dk, dv, dlambda, drms_w, workspace, stream));
+}
+
+int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
+                        const float* dlambda, float* dlq1, float* dlk1, float* dlq2, float* dlk2,
+                        cudaStream_t stream) {
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !dlambda || !dlq1 || !dlk1 || !dlq2 || !dlk2) return DIFFATTN_ERR_INVALID_ARG;
+  if (d < 1 || d > 4096) return DIFFATTN_ERR_INVALID_ARG;
+  return cuda_status(launch_lambda_bwd(lq1, lk1, lq2, lk2, d, dlambda, dlq1, dlk1, dlq2, dlk2, stream));
+}
+
 size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen) {
   return decode_workspace_bytes(S, H, d, max_seqlen);
 }

@@ -41,6 +41,16 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
 cudaError_t launch_quantize_qk(const void* x, int B, int N, int H, int d, void* codes, float* scales,
                                cudaStream_t stream);
 
+// Backward pass of the prefill (CUDA cores; bf16 or fp32 inputs, fp32 gradients).
+size_t bwd_workspace_bytes(int B, int N, int H, int d);
+cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* dy, int bf16, int B, int N, int H,
+                       int d, int causal, const float* lambda, float lambda_init, const float* rms_w, float eps,
+                       int mode, float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
+                       cudaStream_t stream);
+cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
+                              const float* dlambda, float* dlq1, float* dlk1, float* dlq2, float* dlk2,
+                              cudaStream_t stream);
+
 // Split-KV decode (bf16, d = 128).
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,

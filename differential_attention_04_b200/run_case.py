@@ -21,7 +21,7 @@ from .build import build
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kind", choices=["prefill", "decode"])
+    ap.add_argument("kind", choices=["prefill", "decode", "bwd"])
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--H", type=int, default=12)
@@ -56,6 +56,13 @@ def main(argv=None):
         else:
             run = lambda: api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps,
                                            inp.causal, out=y)
+    elif a.kind == "bwd":
+        inp = wl.make_prefill(a.B, a.N, a.H, a.d, causal=bool(a.causal), dtype=a.dtype, seed=a.seed, device=dev)
+        lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+        dy = torch.randn(inp.v.shape, device=dev).to(inp.v.dtype)
+        ws = torch.empty(api.bwd_workspace_size(a.B, a.N, a.H, a.d), dtype=torch.uint8, device=dev)
+        run = lambda: api.diffattn_bwd(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps,
+                                       inp.causal, workspace=ws)
     else:
         inp = wl.make_decode(a.S, a.H, a.d, a.lmin, a.lmax, seed=a.seed, device=dev)
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)

@@ -123,6 +123,47 @@ int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o,
                       float eps, int mode, cudaStream_t stream);
 
 /*
+ * Backward pass (training).  Gradients of diffattn_fwd_mode's output with
+ * respect to q, k, v, lambda and the RMSNorm weight, for an upstream gradient
+ * dy: the derivative of the DiffAttn equation (first page, the section with
+ * the DiffAttn equation; peer review "Differential Transformer", Summary,
+ * Eq. 1) and of the headwise RMSNorm and (1 - lambda_init) scale (Eq. 3).
+ *
+ * diffattn_bwd_workspace_size -- bytes of workspace for diffattn_bwd (0 for
+ *   sizes below 1): fp32 [B, N, H, 2d] plus 16 bytes per (b, n, h).
+ * diffattn_bwd
+ *   q, k, v, dy : as in diffattn_fwd (dy has v's shape), dtype BF16 or F32
+ *   lambda, lambda_init, rms_w, eps, causal, mode : as in diffattn_fwd_mode
+ *   dq, dk      : device float32 [B, N, H, 2, d], written
+ *   dv          : device float32 [B, N, H, 2d], written
+ *   dlambda     : device float32 scalar, written (0 in DIFFATTN_MODE_LAMBDA_ZERO)
+ *   drms_w      : device float32 [2d], written
+ *   workspace   : device, >= diffattn_bwd_workspace_size bytes, 16-byte aligned
+ * CUDA cores (fp32 arithmetic), 1 <= d <= 128.  Stream-ordered; dlambda and
+ * drms_w are summed with atomics, so their last bits may vary from run to run.
+ * Errors: DIFFATTN_ERR_INVALID_ARG, DIFFATTN_ERR_UNSUPPORTED (d > 128),
+ * DIFFATTN_ERR_WORKSPACE, DIFFATTN_ERR_CUDA.
+ */
+size_t diffattn_bwd_workspace_size(int B, int N, int H, int d);
+int diffattn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                 int dtype, int B, int N, int H, int d, int causal,
+                 const float* lambda, float lambda_init, const float* rms_w,
+                 float eps, int mode, float* dq, float* dk, float* dv,
+                 float* dlambda, float* drms_w, void* workspace, size_t ws_bytes,
+                 cudaStream_t stream);
+
+/*
+ * diffattn_lambda_bwd -- gradients of the lambda re-parameterisation (Eq. 2)
+ * for a device dlambda: dlq1 = dlambda e1 lk1, dlk1 = dlambda e1 lq1,
+ * dlq2 = -dlambda e2 lk2, dlk2 = -dlambda e2 lq2, with e1 = exp(lq1 . lk1),
+ * e2 = exp(lq2 . lk2).  All device float32; vectors of length d (1..4096).
+ */
+int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2,
+                        const float* lk2, int d, const float* dlambda,
+                        float* dlq1, float* dlk1, float* dlq2, float* dlk2,
+                        cudaStream_t stream);
+
+/*
  * Low-bit queries and keys (peer review "Differential Transformer",
  * Strengths, the activation-outlier bullet, and Questions, the quantisation
  * bullet: absmax quantisation per logit map and per head).

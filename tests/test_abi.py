@@ -83,6 +83,18 @@ def test_validation_without_gpu(L):
     assert f8(fake, 16, 128, mode=5) == api.ERR_INVALID_ARG
     assert f8(nul, 16, 128) == api.ERR_INVALID_ARG
     assert f8(nul, 0, 128) == api.OK
+    # backward
+    bw = lambda x, N, d, ws, wsb, mode=0: L.diffattn_bwd(x, x, x, x, api.F32, 1, N, 2, d, 1, x, 0.5, x, 1e-5, mode,
+                                                         x, x, x, x, x, ws, wsb, nul)
+    assert bw(fake, 16, 129, fake, 1 << 30) == api.ERR_UNSUPPORTED
+    assert bw(fake, 16, 64, nul, 1 << 30) == api.ERR_WORKSPACE
+    assert bw(fake, 16, 64, fake, 16) == api.ERR_WORKSPACE
+    assert bw(nul, 16, 64, fake, 1 << 30) == api.ERR_INVALID_ARG
+    assert bw(fake, 16, 64, fake, 1 << 30, mode=9) == api.ERR_INVALID_ARG
+    assert bw(fake, 0, 64, fake, 1 << 30) == api.ERR_INVALID_ARG
+    assert L.diffattn_bwd_workspace_size(1, 16, 2, 64) == 4 * 16 * 2 * 128 + 16 * 16 * 2
+    assert L.diffattn_bwd_workspace_size(0, 16, 2, 64) == 0
+    assert L.diffattn_lambda_bwd(nul, nul, nul, nul, 8, nul, nul, nul, nul, nul, nul) == api.ERR_INVALID_ARG
     # decode
     dec = lambda q, d, ws, wsb, S=4: L.diffattn_decode(q, q, q, q, 100, q, S, 2, d, q, 0.5, q, 1e-5, ws, wsb, nul)
     assert dec(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG

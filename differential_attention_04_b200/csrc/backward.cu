@@ -14,7 +14,10 @@
 //   dlambda = (dc/dlambda) <G, A_2 V>
 //
 // Three kernels, each CTA = 8 warps over 32 rows of one (batch, head), tiles
-// of 32 streamed through shared memory (the layout of the fp32 prefill):
+// of 32 streamed through shared memory.  Lane j takes element j of the
+// streamed tile against the warp's own 4 rows (or keys), which sit transposed
+// in shared memory so that one broadcast float4 load feeds 4 FMAs; the
+// gradient sums likewise update 4 rows per loaded operand:
 //   rows:    recompute both maps' online softmax per query row, keeping A_1 V
 //            and A_2 V apart; write G, the two log-sum-exps and D_1, D_2 to
 //            the workspace; reduce dw and dlambda per CTA, then add them.
@@ -73,11 +76,13 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const T* __restrict__ q, 
   extern __shared__ float sm[];
   const int d = a.d, dv = 2 * d, N = a.N, H = a.H;
   const int kstride = (d % 2 == 0) ? d + 1 : d;
-  float* q1s = sm;
-  float* q2s = q1s + kRows * d;
-  float* k1s = q2s + kRows * d;
+  float* q1T = sm;                        // [d][32] this CTA's queries, transposed
+  float* q2T = q1T + d * kRows;
+  float* k1s = q2T + d * kRows;           // [32][kstride] the streamed keys
   float* k2s = k1s + kTile * kstride;
-  float* vs = k2s + kTile * kstride;
+  float* vs = k2s + kTile * kstride;      // [32][2d]
+  const float4* q1T4 = reinterpret_cast<const float4*>(q1T);
+  const float4* q2T4 = reinterpret_cast<const float4*>(q2T);
   const int b = blockIdx.z, h = blockIdx.y, q0 = blockIdx.x * kRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t tok_qk = static_cast<size_t>(H) * 2 * d, tok_v = static_cast<size_t>(H) * dv;
@@ -88,9 +93,9 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const T* __restrict__ q, 
   const float coef = map2_coefficient(mode, *lambda_ptr);
 
   for (int i = threadIdx.x; i < kRows * d; i += blockDim.x) {
-    const int r = i / d, c = i % d, n = q0 + r;
-    q1s[i] = n < N ? ldf(qb + n * tok_qk + c) : 0.f;
-    q2s[i] = n < N ? ldf(qb + n * tok_qk + d + c) : 0.f;
+    const int r = i % kRows, c = i / kRows, n = q0 + r;
+    q1T[i] = n < N ? ldf(qb + n * tok_qk + c) : 0.f;
+    q2T[i] = n < N ? ldf(qb + n * tok_qk + d + c) : 0.f;
   }
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
   float m1[kPerWarp], l1[kPerWarp], m2[kPerWarp], l2[kPerWarp];
@@ -115,29 +120,34 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const T* __restrict__ q, 
       vs[i] = n < N ? ldf(vb + n * tok_v + c) : 0.f;
     }
     __syncthreads();
+    // scores of key kt + lane against the warp's 4 rows, both maps
+    float s1[kPerWarp], s2[kPerWarp];
+#pragma unroll
+    for (int rr = 0; rr < kPerWarp; ++rr) s1[rr] = s2[rr] = 0.f;
+    for (int c = 0; c < d; ++c) {
+      const float ka = k1s[lane * kstride + c], kb2 = k2s[lane * kstride + c];
+      const float4 qa = q1T4[c * (kRows / 4) + warp], qb4 = q2T4[c * (kRows / 4) + warp];
+      s1[0] = fmaf(qa.x, ka, s1[0]); s1[1] = fmaf(qa.y, ka, s1[1]);
+      s1[2] = fmaf(qa.z, ka, s1[2]); s1[3] = fmaf(qa.w, ka, s1[3]);
+      s2[0] = fmaf(qb4.x, kb2, s2[0]); s2[1] = fmaf(qb4.y, kb2, s2[1]);
+      s2[2] = fmaf(qb4.z, kb2, s2[2]); s2[3] = fmaf(qb4.w, kb2, s2[3]);
+    }
+    const int j = kt + lane;
+    float p1[kPerWarp], p2[kPerWarp];
 #pragma unroll
     for (int rr = 0; rr < kPerWarp; ++rr) {
-      const int r = warp * kPerWarp + rr, qi = q0 + r;
-      if (qi >= N) continue;
-      const int j = kt + lane;
-      const bool valid = j < N && (!a.causal || j <= qi);
-      float s1 = -INFINITY, s2 = -INFINITY;
-      if (valid) {
-        float a1 = 0.f, a2 = 0.f;
-        for (int c = 0; c < d; ++c) {
-          a1 = fmaf(q1s[r * d + c], k1s[lane * kstride + c], a1);
-          a2 = fmaf(q2s[r * d + c], k2s[lane * kstride + c], a2);
-        }
-        s1 = a1 * scale;
-        s2 = a2 * scale;
-      }
-      const float t1 = warp_max(s1), t2 = warp_max(s2);
-      if (t1 == -INFINITY) continue;  // no visible key in this tile (both maps share the mask)
+      const int qi = q0 + warp * kPerWarp + rr;
+      const bool valid = qi < N && j < N && (!a.causal || j <= qi);
+      const float v1 = valid ? s1[rr] * scale : -INFINITY, v2 = valid ? s2[rr] * scale : -INFINITY;
+      const float t1 = warp_max(v1), t2 = warp_max(v2);
+      p1[rr] = p2[rr] = 0.f;
+      if (t1 == -INFINITY) continue;  // this row sees no key of the tile (both maps share the mask)
       const float mn1 = fmaxf(m1[rr], t1), mn2 = fmaxf(m2[rr], t2);
       const float al1 = expf(m1[rr] - mn1), al2 = expf(m2[rr] - mn2);
-      const float p1 = valid ? expf(s1 - mn1) : 0.f, p2 = valid ? expf(s2 - mn2) : 0.f;
-      l1[rr] = l1[rr] * al1 + warp_sum(p1);
-      l2[rr] = l2[rr] * al2 + warp_sum(p2);
+      p1[rr] = valid ? expf(v1 - mn1) : 0.f;
+      p2[rr] = valid ? expf(v2 - mn2) : 0.f;
+      l1[rr] = l1[rr] * al1 + warp_sum(p1[rr]);
+      l2[rr] = l2[rr] * al2 + warp_sum(p2[rr]);
       m1[rr] = mn1;
       m2[rr] = mn2;
 #pragma unroll
@@ -145,16 +155,24 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const T* __restrict__ q, 
         o1[rr][u] *= al1;
         o2[rr][u] *= al2;
       }
-      const int jn = min(kTile, N - kt);
-      for (int jj = 0; jj < jn; ++jj) {
-        const float pj1 = __shfl_sync(0xffffffffu, p1, jj), pj2 = __shfl_sync(0xffffffffu, p2, jj);
+    }
+    const int jn = min(kTile, N - kt);
+    for (int jj = 0; jj < jn; ++jj) {
+      float pj1[kPerWarp], pj2[kPerWarp];
 #pragma unroll
-        for (int u = 0; u < kMaxU; ++u) {
-          const int c = lane + 32 * u;
-          if (c < dv) {
-            const float vv = vs[jj * dv + c];
-            o1[rr][u] = fmaf(pj1, vv, o1[rr][u]);
-            o2[rr][u] = fmaf(pj2, vv, o2[rr][u]);
+      for (int rr = 0; rr < kPerWarp; ++rr) {
+        pj1[rr] = __shfl_sync(0xffffffffu, p1[rr], jj);
+        pj2[rr] = __shfl_sync(0xffffffffu, p2[rr], jj);
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxU; ++u) {
+        const int c = lane + 32 * u;
+        if (c < dv) {
+          const float vv = vs[jj * dv + c];
+#pragma unroll
+          for (int rr = 0; rr < kPerWarp; ++rr) {
+            o1[rr][u] = fmaf(pj1[rr], vv, o1[rr][u]);
+            o2[rr][u] = fmaf(pj2[rr], vv, o2[rr][u]);
           }
         }
       }
@@ -239,13 +257,16 @@ __global__ void __launch_bounds__(256) bwd_keys_kernel(const T* __restrict__ q, 
   const int d = a.d, dv = 2 * d, N = a.N, H = a.H;
   const int qstride = (d % 2 == 0) ? d + 1 : d;
   const int gstride = dv + 1;
-  float* k1s = sm;                        // [32][d]   this CTA's keys
-  float* k2s = k1s + kRows * d;
-  float* vs = k2s + kRows * d;            // [32][2d]
-  float* q1s = vs + kRows * dv;           // [32][qstride] the streamed queries
+  float* k1T = sm;                        // [d][32]  this CTA's keys, transposed
+  float* k2T = k1T + d * kRows;
+  float* vT = k2T + d * kRows;            // [2d][32]
+  float* q1s = vT + dv * kRows;           // [32][qstride] the streamed queries
   float* q2s = q1s + kTile * qstride;
   float* gs = q2s + kTile * qstride;      // [32][gstride]
   float4* st = reinterpret_cast<float4*>(gs + kTile * gstride);  // [32]
+  const float4* k1T4 = reinterpret_cast<const float4*>(k1T);
+  const float4* k2T4 = reinterpret_cast<const float4*>(k2T);
+  const float4* vT4 = reinterpret_cast<const float4*>(vT);
   const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * kRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t tok_qk = static_cast<size_t>(H) * 2 * d, tok_v = static_cast<size_t>(H) * dv;
@@ -256,13 +277,13 @@ __global__ void __launch_bounds__(256) bwd_keys_kernel(const T* __restrict__ q, 
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
 
   for (int i = threadIdx.x; i < kRows * d; i += blockDim.x) {
-    const int r = i / d, c = i % d, n = k0 + r;
-    k1s[i] = n < N ? ldf(kb + n * tok_qk + c) : 0.f;
-    k2s[i] = n < N ? ldf(kb + n * tok_qk + d + c) : 0.f;
+    const int r = i % kRows, c = i / kRows, n = k0 + r;
+    k1T[i] = n < N ? ldf(kb + n * tok_qk + c) : 0.f;
+    k2T[i] = n < N ? ldf(kb + n * tok_qk + d + c) : 0.f;
   }
   for (int i = threadIdx.x; i < kRows * dv; i += blockDim.x) {
-    const int r = i / dv, c = i % dv, n = k0 + r;
-    vs[i] = n < N ? ldf(vb + n * tok_v + c) : 0.f;
+    const int r = i % kRows, c = i / kRows, n = k0 + r;
+    vT[i] = n < N ? ldf(vb + n * tok_v + c) : 0.f;
   }
   float dk1[kPerWarp][kMaxD], dk2[kPerWarp][kMaxD], dvacc[kPerWarp][kMaxU];
 #pragma unroll
@@ -272,8 +293,9 @@ __global__ void __launch_bounds__(256) bwd_keys_kernel(const T* __restrict__ q, 
 #pragma unroll
     for (int u = 0; u < kMaxU; ++u) dvacc[kk][u] = 0.f;
   }
-  const int qstart = a.causal ? k0 : 0;  // causal: queries before this key tile see none of its keys
-  for (int qt = qstart - (qstart % kTile); qt < N; qt += kTile) {
+  const int kw = k0 + warp * kPerWarp;   // the warp's first key
+  // causal: queries before this key tile see none of its keys (k0 is a multiple of the tile)
+  for (int qt = a.causal ? k0 : 0; qt < N; qt += kTile) {
     __syncthreads();
     for (int i = threadIdx.x; i < kTile * d; i += blockDim.x) {
       const int j = i / d, c = i % d, n = qt + j;
@@ -289,50 +311,72 @@ __global__ void __launch_bounds__(256) bwd_keys_kernel(const T* __restrict__ q, 
       st[j] = n < N ? a.stats[(static_cast<size_t>(b) * N + n) * H + h] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
+    // query qt + lane against the warp's 4 keys: scores of both maps and G . V
+    float s1[kPerWarp], s2[kPerWarp], vg[kPerWarp];
+#pragma unroll
+    for (int kk = 0; kk < kPerWarp; ++kk) s1[kk] = s2[kk] = vg[kk] = 0.f;
+    for (int c = 0; c < d; ++c) {
+      const float qa = q1s[lane * qstride + c], qb2 = q2s[lane * qstride + c];
+      const float4 ka = k1T4[c * (kRows / 4) + warp], kb4 = k2T4[c * (kRows / 4) + warp];
+      s1[0] = fmaf(ka.x, qa, s1[0]); s1[1] = fmaf(ka.y, qa, s1[1]);
+      s1[2] = fmaf(ka.z, qa, s1[2]); s1[3] = fmaf(ka.w, qa, s1[3]);
+      s2[0] = fmaf(kb4.x, qb2, s2[0]); s2[1] = fmaf(kb4.y, qb2, s2[1]);
+      s2[2] = fmaf(kb4.z, qb2, s2[2]); s2[3] = fmaf(kb4.w, qb2, s2[3]);
+    }
+    for (int c = 0; c < dv; ++c) {
+      const float gv = gs[lane * gstride + c];
+      const float4 v4 = vT4[c * (kRows / 4) + warp];
+      vg[0] = fmaf(v4.x, gv, vg[0]); vg[1] = fmaf(v4.y, gv, vg[1]);
+      vg[2] = fmaf(v4.z, gv, vg[2]); vg[3] = fmaf(v4.w, gv, vg[3]);
+    }
+    const int qi = qt + lane;
+    const float4 s4 = st[lane];
+    float ds1[kPerWarp], ds2[kPerWarp], pv[kPerWarp];
 #pragma unroll
     for (int kk = 0; kk < kPerWarp; ++kk) {
-      const int r = warp * kPerWarp + kk, kj = k0 + r;
-      if (kj >= N) continue;
-      const int qi = qt + lane;
-      const bool valid = qi < N && (!a.causal || qi >= kj);
-      float p1 = 0.f, p2 = 0.f, ds1 = 0.f, ds2 = 0.f;
-      if (valid) {
-        float a1 = 0.f, a2 = 0.f, vg = 0.f;
-        for (int c = 0; c < d; ++c) {
-          a1 = fmaf(k1s[r * d + c], q1s[lane * qstride + c], a1);
-          a2 = fmaf(k2s[r * d + c], q2s[lane * qstride + c], a2);
-        }
-        for (int c = 0; c < dv; ++c) vg = fmaf(vs[r * dv + c], gs[lane * gstride + c], vg);
-        const float4 s4 = st[lane];
-        p1 = expf(a1 * scale - s4.x);
-        p2 = expf(a2 * scale - s4.y);
-        ds1 = p1 * (vg - s4.z);
-        ds2 = p2 * (coef * vg - s4.w);
-      }
-      const float pv = p1 + coef * p2;  // dV gets (A_1 + c A_2)^T G
-      const int jn = min(kTile, N - qt);
-      for (int jj = 0; jj < jn; ++jj) {
-        const float pvj = __shfl_sync(0xffffffffu, pv, jj);
-        const float d1j = __shfl_sync(0xffffffffu, ds1, jj), d2j = __shfl_sync(0xffffffffu, ds2, jj);
+      const int kj = kw + kk;
+      const bool valid = qi < N && kj < N && (!a.causal || qi >= kj);
+      const float p1 = valid ? expf(s1[kk] * scale - s4.x) : 0.f;
+      const float p2 = valid ? expf(s2[kk] * scale - s4.y) : 0.f;
+      ds1[kk] = p1 * (vg[kk] - s4.z);
+      ds2[kk] = p2 * (coef * vg[kk] - s4.w);
+      pv[kk] = p1 + coef * p2;  // dV gets (A_1 + c A_2)^T G
+    }
+    const int jn = min(kTile, N - qt);
+    for (int jj = 0; jj < jn; ++jj) {
+      float d1[kPerWarp], d2[kPerWarp], pj[kPerWarp];
 #pragma unroll
-        for (int u = 0; u < kMaxD; ++u) {
-          const int c = lane + 32 * u;
-          if (c < d) {
-            dk1[kk][u] = fmaf(d1j, q1s[jj * qstride + c], dk1[kk][u]);
-            dk2[kk][u] = fmaf(d2j, q2s[jj * qstride + c], dk2[kk][u]);
+      for (int kk = 0; kk < kPerWarp; ++kk) {
+        d1[kk] = __shfl_sync(0xffffffffu, ds1[kk], jj);
+        d2[kk] = __shfl_sync(0xffffffffu, ds2[kk], jj);
+        pj[kk] = __shfl_sync(0xffffffffu, pv[kk], jj);
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxD; ++u) {
+        const int c = lane + 32 * u;
+        if (c < d) {
+          const float qa = q1s[jj * qstride + c], qb2 = q2s[jj * qstride + c];
+#pragma unroll
+          for (int kk = 0; kk < kPerWarp; ++kk) {
+            dk1[kk][u] = fmaf(d1[kk], qa, dk1[kk][u]);
+            dk2[kk][u] = fmaf(d2[kk], qb2, dk2[kk][u]);
           }
         }
+      }
 #pragma unroll
-        for (int u = 0; u < kMaxU; ++u) {
-          const int c = lane + 32 * u;
-          if (c < dv) dvacc[kk][u] = fmaf(pvj, gs[jj * gstride + c], dvacc[kk][u]);
+      for (int u = 0; u < kMaxU; ++u) {
+        const int c = lane + 32 * u;
+        if (c < dv) {
+          const float gv = gs[jj * gstride + c];
+#pragma unroll
+          for (int kk = 0; kk < kPerWarp; ++kk) dvacc[kk][u] = fmaf(pj[kk], gv, dvacc[kk][u]);
         }
       }
     }
   }
 #pragma unroll
   for (int kk = 0; kk < kPerWarp; ++kk) {
-    const int kj = k0 + warp * kPerWarp + kk;
+    const int kj = kw + kk;
     if (kj >= N) continue;
     const size_t row = (static_cast<size_t>(b) * N + kj) * H + h;
 #pragma unroll
@@ -361,12 +405,15 @@ __global__ void __launch_bounds__(256) bwd_queries_kernel(const T* __restrict__ 
   const int d = a.d, dv = 2 * d, N = a.N, H = a.H;
   const int kstride = (d % 2 == 0) ? d + 1 : d;
   const int vstride = dv + 1;
-  float* q1s = sm;                       // [32][d]   this CTA's queries
-  float* q2s = q1s + kRows * d;
-  float* gs = q2s + kRows * d;           // [32][2d]
-  float* k1s = gs + kRows * dv;          // [32][kstride] the streamed keys
+  float* q1T = sm;                       // [d][32]  this CTA's queries, transposed
+  float* q2T = q1T + d * kRows;
+  float* gT = q2T + d * kRows;           // [2d][32]
+  float* k1s = gT + dv * kRows;          // [32][kstride] the streamed keys
   float* k2s = k1s + kTile * kstride;
   float* vs = k2s + kTile * kstride;     // [32][vstride]
+  const float4* q1T4 = reinterpret_cast<const float4*>(q1T);
+  const float4* q2T4 = reinterpret_cast<const float4*>(q2T);
+  const float4* gT4 = reinterpret_cast<const float4*>(gT);
   const int b = blockIdx.z, h = blockIdx.y, q0 = blockIdx.x * kRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t tok_qk = static_cast<size_t>(H) * 2 * d, tok_v = static_cast<size_t>(H) * dv;
@@ -377,18 +424,19 @@ __global__ void __launch_bounds__(256) bwd_queries_kernel(const T* __restrict__ 
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
 
   for (int i = threadIdx.x; i < kRows * d; i += blockDim.x) {
-    const int r = i / d, c = i % d, n = q0 + r;
-    q1s[i] = n < N ? ldf(qb + n * tok_qk + c) : 0.f;
-    q2s[i] = n < N ? ldf(qb + n * tok_qk + d + c) : 0.f;
+    const int r = i % kRows, c = i / kRows, n = q0 + r;
+    q1T[i] = n < N ? ldf(qb + n * tok_qk + c) : 0.f;
+    q2T[i] = n < N ? ldf(qb + n * tok_qk + d + c) : 0.f;
   }
   for (int i = threadIdx.x; i < kRows * dv; i += blockDim.x) {
-    const int r = i / dv, c = i % dv, n = q0 + r;
-    gs[i] = n < N ? a.G[((static_cast<size_t>(b) * N + n) * H + h) * dv + c] : 0.f;
+    const int r = i % kRows, c = i / kRows, n = q0 + r;
+    gT[i] = n < N ? a.G[((static_cast<size_t>(b) * N + n) * H + h) * dv + c] : 0.f;
   }
+  const int qw = q0 + warp * kPerWarp;   // the warp's first query row
   float4 srow[kPerWarp];
 #pragma unroll
   for (int rr = 0; rr < kPerWarp; ++rr) {
-    const int n = q0 + warp * kPerWarp + rr;
+    const int n = qw + rr;
     srow[rr] = n < N ? a.stats[(static_cast<size_t>(b) * N + n) * H + h] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   float dq1[kPerWarp][kMaxD], dq2[kPerWarp][kMaxD];
@@ -409,33 +457,52 @@ __global__ void __launch_bounds__(256) bwd_queries_kernel(const T* __restrict__ 
       vs[j * vstride + c] = n < N ? ldf(vb + n * tok_v + c) : 0.f;
     }
     __syncthreads();
+    // key kt + lane against the warp's 4 rows: scores of both maps and G . V
+    float s1[kPerWarp], s2[kPerWarp], vg[kPerWarp];
+#pragma unroll
+    for (int rr = 0; rr < kPerWarp; ++rr) s1[rr] = s2[rr] = vg[rr] = 0.f;
+    for (int c = 0; c < d; ++c) {
+      const float ka = k1s[lane * kstride + c], kb2 = k2s[lane * kstride + c];
+      const float4 qa = q1T4[c * (kRows / 4) + warp], qb4 = q2T4[c * (kRows / 4) + warp];
+      s1[0] = fmaf(qa.x, ka, s1[0]); s1[1] = fmaf(qa.y, ka, s1[1]);
+      s1[2] = fmaf(qa.z, ka, s1[2]); s1[3] = fmaf(qa.w, ka, s1[3]);
+      s2[0] = fmaf(qb4.x, kb2, s2[0]); s2[1] = fmaf(qb4.y, kb2, s2[1]);
+      s2[2] = fmaf(qb4.z, kb2, s2[2]); s2[3] = fmaf(qb4.w, kb2, s2[3]);
+    }
+    for (int c = 0; c < dv; ++c) {
+      const float vv = vs[lane * vstride + c];
+      const float4 g4 = gT4[c * (kRows / 4) + warp];
+      vg[0] = fmaf(g4.x, vv, vg[0]); vg[1] = fmaf(g4.y, vv, vg[1]);
+      vg[2] = fmaf(g4.z, vv, vg[2]); vg[3] = fmaf(g4.w, vv, vg[3]);
+    }
+    const int kj = kt + lane;
+    float ds1[kPerWarp], ds2[kPerWarp];
 #pragma unroll
     for (int rr = 0; rr < kPerWarp; ++rr) {
-      const int r = warp * kPerWarp + rr, qi = q0 + r;
-      if (qi >= N) continue;
-      const int kj = kt + lane;
-      const bool valid = kj < N && (!a.causal || kj <= qi);
-      float ds1 = 0.f, ds2 = 0.f;
-      if (valid) {
-        float a1 = 0.f, a2 = 0.f, vg = 0.f;
-        for (int c = 0; c < d; ++c) {
-          a1 = fmaf(q1s[r * d + c], k1s[lane * kstride + c], a1);
-          a2 = fmaf(q2s[r * d + c], k2s[lane * kstride + c], a2);
-        }
-        for (int c = 0; c < dv; ++c) vg = fmaf(gs[r * dv + c], vs[lane * vstride + c], vg);
-        const float p1 = expf(a1 * scale - srow[rr].x), p2 = expf(a2 * scale - srow[rr].y);
-        ds1 = p1 * (vg - srow[rr].z);
-        ds2 = p2 * (coef * vg - srow[rr].w);
-      }
-      const int jn = min(kTile, N - kt);
-      for (int jj = 0; jj < jn; ++jj) {
-        const float d1j = __shfl_sync(0xffffffffu, ds1, jj), d2j = __shfl_sync(0xffffffffu, ds2, jj);
+      const int qi = qw + rr;
+      const bool valid = qi < N && kj < N && (!a.causal || kj <= qi);
+      const float p1 = valid ? expf(s1[rr] * scale - srow[rr].x) : 0.f;
+      const float p2 = valid ? expf(s2[rr] * scale - srow[rr].y) : 0.f;
+      ds1[rr] = p1 * (vg[rr] - srow[rr].z);
+      ds2[rr] = p2 * (coef * vg[rr] - srow[rr].w);
+    }
+    const int jn = min(kTile, N - kt);
+    for (int jj = 0; jj < jn; ++jj) {
+      float d1[kPerWarp], d2[kPerWarp];
 #pragma unroll
-        for (int u = 0; u < kMaxD; ++u) {
-          const int c = lane + 32 * u;
-          if (c < d) {
-            dq1[rr][u] = fmaf(d1j, k1s[jj * kstride + c], dq1[rr][u]);
-            dq2[rr][u] = fmaf(d2j, k2s[jj * kstride + c], dq2[rr][u]);
+      for (int rr = 0; rr < kPerWarp; ++rr) {
+        d1[rr] = __shfl_sync(0xffffffffu, ds1[rr], jj);
+        d2[rr] = __shfl_sync(0xffffffffu, ds2[rr], jj);
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxD; ++u) {
+        const int c = lane + 32 * u;
+        if (c < d) {
+          const float ka = k1s[jj * kstride + c], kb2 = k2s[jj * kstride + c];
+#pragma unroll
+          for (int rr = 0; rr < kPerWarp; ++rr) {
+            dq1[rr][u] = fmaf(d1[rr], ka, dq1[rr][u]);
+            dq2[rr][u] = fmaf(d2[rr], kb2, dq2[rr][u]);
           }
         }
       }
@@ -443,7 +510,7 @@ __global__ void __launch_bounds__(256) bwd_queries_kernel(const T* __restrict__ 
   }
 #pragma unroll
   for (int rr = 0; rr < kPerWarp; ++rr) {
-    const int qi = q0 + warp * kPerWarp + rr;
+    const int qi = qw + rr;
     if (qi >= N) continue;
     const size_t row = (static_cast<size_t>(b) * N + qi) * H + h;
 #pragma unroll

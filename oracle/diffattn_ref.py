@@ -219,11 +219,12 @@ def diffattn_fwd(q, k, v, lam: float, lambda_init: float, w, eps: float, causal:
     return y
 
 
-def decode_head_prenorm(q1, q2, k1, k2, v, lam: float) -> np.ndarray:
+def decode_head_prenorm(q1, q2, k1, k2, v, lam: float, mode: str = "diff") -> np.ndarray:
     """DiffAttn for one query (length-1 decode) against L cached keys.
 
     q1, q2 : [d]; k1, k2 : [L, d]; v : [L, 2d]  ->  O : [2d].  The query sees
-    all L keys (its own included), so no mask applies.
+    all L keys (its own included), so no mask applies.  ``mode`` selects the
+    combination of the two maps (see MODES).
     """
     q1 = np.asarray(q1, dtype=np.float64)[None, :]
     q2 = np.asarray(q2, dtype=np.float64)[None, :]
@@ -231,12 +232,12 @@ def decode_head_prenorm(q1, q2, k1, k2, v, lam: float) -> np.ndarray:
     k2 = np.asarray(k2, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     scale = 1.0 / math.sqrt(q1.shape[1])
-    D = diff_weights((q1 @ k1.T) * scale, (q2 @ k2.T) * scale, lam)
+    D = map_weights((q1 @ k1.T) * scale, (q2 @ k2.T) * scale, lam, mode)
     return (D @ v)[0]
 
 
 def diffattn_decode(q, k_cache, v_cache, cu_seqlens, lam: float, lambda_init: float, w,
-                    eps: float, pairs=None) -> np.ndarray:
+                    eps: float, pairs=None, mode: str = "diff") -> np.ndarray:
     """Decode over a packed KV cache: normalised output per (sequence, head).
 
     q : [S, H, 2, d]; k_cache : [T, H, 2, d]; v_cache : [T, H, 2d];
@@ -252,6 +253,6 @@ def diffattn_decode(q, k_cache, v_cache, cu_seqlens, lam: float, lambda_init: fl
         lo, hi = int(cu[s]), int(cu[s + 1])
         kc = np.asarray(k_cache[lo:hi, h], dtype=np.float64)
         vc = np.asarray(v_cache[lo:hi, h], dtype=np.float64)
-        O = decode_head_prenorm(q[s, h, 0], q[s, h, 1], kc[:, 0], kc[:, 1], vc, lam)
+        O = decode_head_prenorm(q[s, h, 0], q[s, h, 1], kc[:, 0], kc[:, 1], vc, lam, mode)
         y[s, h] = headwise_rmsnorm(O, w, eps, lambda_init)
     return y

@@ -206,13 +206,16 @@ def pin_decode_is_last_prefill_row():
     qs = rng.standard_normal((len(lens), H, 2, d))
     w = 1 + 0.1 * rng.standard_normal(2 * d)
     lam, lam_init, eps = 0.31, 0.5, 1e-5
-    y = ref.diffattn_decode(qs, kc, vc, cu, lam, lam_init, w, eps)
-    for s, L in enumerate(lens):
-        lo = cu[s]
-        q = rng.standard_normal((1, L, H, 2, d))
-        q[0, L - 1] = qs[s]
-        yp = ref.diffattn_fwd(q, kc[None, lo:lo + L], vc[None, lo:lo + L], lam, lam_init, w, eps, True)
-        assert np.allclose(y[s], yp[0, L - 1], atol=1e-12)
+    qp = [rng.standard_normal((1, L, H, 2, d)) for L in lens]
+    for mode in ref.MODES:  # in every combination mode
+        y = ref.diffattn_decode(qs, kc, vc, cu, lam, lam_init, w, eps, mode=mode)
+        for s, L in enumerate(lens):
+            lo = cu[s]
+            q = qp[s].copy()
+            q[0, L - 1] = qs[s]
+            yp = ref.diffattn_fwd(q, kc[None, lo:lo + L], vc[None, lo:lo + L], lam, lam_init, w, eps, True,
+                                  mode=mode)
+            assert np.allclose(y[s], yp[0, L - 1], atol=1e-12)
 
 
 def pin_sampled_rows():
@@ -362,8 +365,8 @@ def _mut_zero_keeps_map2(S1, S2, lam, mode="diff"):
     return ref.softmax_rows(S1) - float(lam) * ref.softmax_rows(S2)
 
 
-def _mut_decode_maps(q1, q2, k1, k2, v, lam):
-    return _orig_decode(q1, q2, k1, k1, v, lam)
+def _mut_decode_maps(q1, q2, k1, k2, v, lam, mode="diff"):
+    return _orig_decode(q1, q2, k1, k1, v, lam, mode)
 
 
 _orig_head = ref.diffattn_head_prenorm

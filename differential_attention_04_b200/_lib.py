@@ -31,6 +31,8 @@ SIGNATURES = {
     "diffattn_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _c_float,
                                  _vp, _c_float, _vp, _c_size, _vp]),
+    "diffattn_decode_mode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _c_float,
+                                      _vp, _c_float, _c_int, _vp, _c_size, _vp]),
     "diffattn_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp,
                                          _c_float, _vp, _c_float, _vp]),
     "diffattn_device_status": (_c_int, [ctypes.POINTER(_c_int)]),

@@ -177,8 +177,9 @@ def decode_workspace_size(S: int, H: int, d: int, max_seqlen: int) -> int:
 def diffattn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, cu_seqlens: torch.Tensor,
                     max_seqlen: int, lam: torch.Tensor, lambda_init: float, rms_w: torch.Tensor,
                     eps: float = 1e-5, workspace: torch.Tensor | None = None,
-                    out: torch.Tensor | None = None) -> torch.Tensor:
-    """Decode.  q: [S, H, 2, d]; k_cache: [T, H, 2, d]; v_cache: [T, H, 2d]; cu_seqlens: int32 [S + 1]."""
+                    out: torch.Tensor | None = None, mode: int = MODE_DIFF) -> torch.Tensor:
+    """Decode.  q: [S, H, 2, d]; k_cache: [T, H, 2, d]; v_cache: [T, H, 2d]; cu_seqlens: int32 [S + 1].
+    ``mode`` as in diffattn_fwd."""
     _dev(q, k_cache, v_cache, cu_seqlens, lam, rms_w)
     S, H, two, d = q.shape
     if cu_seqlens.dtype != torch.int32 or cu_seqlens.numel() != S + 1:
@@ -188,10 +189,16 @@ def diffattn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty((S, H, 2 * d), dtype=q.dtype, device=q.device)
-    _check("diffattn_decode", lib().diffattn_decode(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
-        _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _ptr(workspace), workspace.numel(),
-        _stream()))
+    if mode == MODE_DIFF:
+        _check("diffattn_decode", lib().diffattn_decode(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
+            _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _ptr(workspace), workspace.numel(),
+            _stream()))
+    else:
+        _check("diffattn_decode_mode", lib().diffattn_decode_mode(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
+            _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode), _ptr(workspace), workspace.numel(),
+            _stream()))
     return out
 
 

@@ -238,7 +238,17 @@ size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen) {
 int diffattn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens, int max_seqlen,
                     void* o, int S, int H, int d, const float* lambda, float lambda_init, const float* rms_w,
                     float eps, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return diffattn_decode_mode(q, k_cache, v_cache, cu_seqlens, max_seqlen, o, S, H, d, lambda, lambda_init, rms_w,
+                              eps, DIFFATTN_MODE_DIFF, workspace, ws_bytes, stream);
+}
+
+int diffattn_decode_mode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
+                         int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
+                         const float* rms_w, float eps, int mode, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream) {
   if (S < 1 || H < 1 || d < 1 || max_seqlen < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
   if (!q || !k_cache || !v_cache || !cu_seqlens || !o || !lambda || !rms_w) return DIFFATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
     return DIFFATTN_ERR_INVALID_ARG;
@@ -247,7 +257,7 @@ int diffattn_decode(const void* q, const void* k_cache, const void* v_cache, con
   const size_t need = decode_workspace_bytes(S, H, d, max_seqlen);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
   return cuda_status(launch_decode(q, k_cache, v_cache, cu_seqlens, max_seqlen, o, S, H, d, lambda, lambda_init,
-                                   rms_w, eps, workspace, stream));
+                                   rms_w, eps, mode, workspace, stream));
 }
 
 }  // extern "C"

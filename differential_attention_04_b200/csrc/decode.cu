@@ -215,8 +215,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
 __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __restrict__ ws,
                                                              const int* __restrict__ cu_seqlens, int max_seqlen,
                                                              int H, int max_chunks, __nv_bfloat16* __restrict__ o,
-                                                             const float* __restrict__ lambda_ptr, float lambda_init,
-                                                             const float* __restrict__ rms_w, float eps) {
+                                                             const float* __restrict__ lambda_ptr, int mode,
+                                                             float lambda_init, const float* __restrict__ rms_w,
+                                                             float eps) {
   const int h = blockIdx.x, s = blockIdx.y;
   const int c = threadIdx.x;
   const int L = min(cu_seqlens[s + 1] - cu_seqlens[s], max_seqlen);
@@ -236,8 +237,7 @@ __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __rest
     O1 = fmaf(f1, r[4 + c], O1);
     O2 = fmaf(f2, r[4 + kDV + c], O2);
   }
-  const float lam = *lambda_ptr;
-  const float ov = O1 / L1 - lam * (O2 / L2);
+  const float ov = O1 / L1 + map2_coefficient(mode, *lambda_ptr) * (O2 / L2);  // c = -lambda, 0 or +lambda
   // sum of squares over the 256 channels
   __shared__ float red[kDV / 32];
   float ss = ov * ov;
@@ -260,7 +260,7 @@ size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen) {
 
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
                           int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
-                          const float* rms_w, float eps, void* workspace, cudaStream_t stream) {
+                          const float* rms_w, float eps, int mode, void* workspace, cudaStream_t stream) {
   (void)d;
   const int max_chunks = (max_seqlen + kChunk - 1) / kChunk;
   dim3 grid(max_chunks, H, S);
@@ -272,7 +272,7 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
   if (e != cudaSuccess) return e;
   decode_combine_kernel<<<dim3(H, S), kDV, 0, stream>>>(static_cast<const float*>(workspace), cu_seqlens,
                                                         max_seqlen, H, max_chunks, static_cast<__nv_bfloat16*>(o),
-                                                        lambda, lambda_init, rms_w, eps);
+                                                        lambda, mode, lambda_init, rms_w, eps);
   return cudaGetLastError();
 }
 

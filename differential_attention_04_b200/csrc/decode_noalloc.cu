@@ -73,7 +73,7 @@ extern "C" int diffattn_decode_noalloc(const void* q, const void* k_cache, const
   // The decode kernels write every scratch entry they later read, so the
   // array needs no clearing between calls.
   return diffattn::launch_decode(q, k_cache, v_cache, cu_seqlens, max_seqlen, o, S, H, d, lambda, lambda_init,
-                                 rms_w, eps, scratch, stream) == cudaSuccess
+                                 rms_w, eps, DIFFATTN_MODE_DIFF, scratch, stream) == cudaSuccess
              ? DIFFATTN_OK
              : DIFFATTN_ERR_CUDA;
 }

@@ -55,6 +55,6 @@ cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* l
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
                           int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
-                          const float* rms_w, float eps, void* workspace, cudaStream_t stream);
+                          const float* rms_w, float eps, int mode, void* workspace, cudaStream_t stream);
 
 }  // namespace diffattn

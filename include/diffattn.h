@@ -239,6 +239,18 @@ int diffattn_decode(const void* q, const void* k_cache, const void* v_cache,
                     size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * diffattn_decode_mode -- diffattn_decode with the combination of the two
+ * maps chosen by `mode` (a diffattn_mode, as in diffattn_fwd_mode).  Other
+ * arguments, layouts and errors are those of diffattn_decode; an unknown mode
+ * gives DIFFATTN_ERR_INVALID_ARG.
+ */
+int diffattn_decode_mode(const void* q, const void* k_cache, const void* v_cache,
+                         const int* cu_seqlens, int max_seqlen, void* o, int S,
+                         int H, int d, const float* lambda, float lambda_init,
+                         const float* rms_w, float eps, int mode, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/*
  * diffattn_decode_noalloc -- diffattn_decode for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is a
  * deployment variant of the same computation, with the same arguments as

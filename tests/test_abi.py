@@ -102,6 +102,9 @@ def test_validation_without_gpu(L):
     assert dec(fake, 128, nul, 1 << 30) == api.ERR_WORKSPACE
     assert dec(fake, 128, fake, 16) == api.ERR_WORKSPACE
     assert dec(fake, 128, fake, 1 << 30, S=0) == api.ERR_INVALID_ARG
+    decm = lambda mode: L.diffattn_decode_mode(fake, fake, fake, fake, 100, fake, 4, 2, 128, fake, 0.5, fake, 1e-5,
+                                               mode, fake, 1 << 30, nul)
+    assert decm(3) == api.ERR_INVALID_ARG and decm(-1) == api.ERR_INVALID_ARG
 
 
 def test_workspace_size(L):

@@ -269,15 +269,15 @@ def test_full_size_64k_needle_sampled():
 
 # ------------------------------------------------------------------ decode --
 
-def run_decode(inp):
+def run_decode(inp, mode=api.MODE_DIFF):
     lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
     y = api.diffattn_decode(inp.q, inp.k_cache, inp.v_cache, inp.cu_seqlens, inp.max_seqlen, lam,
-                            inp.lambda_init, inp.rms_w, inp.eps)
+                            inp.lambda_init, inp.rms_w, inp.eps, mode=mode)
     torch.cuda.synchronize()
     return y
 
 
-def oracle_decode(inp, pairs):
+def oracle_decode(inp, pairs, mode="diff"):
     f = wl.to_f64
     lam = ref.lambda_reparam(f(inp.lq1), f(inp.lk1), f(inp.lq2), f(inp.lk2), inp.lambda_init)
     cu = inp.cu_seqlens.cpu().numpy()
@@ -287,7 +287,7 @@ def oracle_decode(inp, pairs):
         kc = f(inp.k_cache[lo:hi, h:h + 1])
         vc = f(inp.v_cache[lo:hi, h:h + 1])
         out[(s, h)] = ref.diffattn_decode(f(inp.q[s:s + 1, h:h + 1]), kc, vc, [0, hi - lo], lam,
-                                          inp.lambda_init, f(inp.rms_w), inp.eps)[0, 0]
+                                          inp.lambda_init, f(inp.rms_w), inp.eps, mode=mode)[0, 0]
     return out
 
 
@@ -295,6 +295,15 @@ def test_decode_small_full():
     inp = wl.make_decode(7, 3, 128, 0, 0, seqlens=[1, 2, 7, 511, 512, 513, 1500], seed=4, device="cuda")
     y = run_decode(inp)
     want = oracle_decode(inp, [(s, h) for s in range(7) for h in range(3)])
+    got = np.stack([wl.to_f64(y[s, h]) for (s, h) in want])
+    assert_close(got, np.stack(list(want.values())))
+
+
+@pytest.mark.parametrize("mode,name", [(1, "lambda_zero"), (2, "sum")])
+def test_decode_control_modes(mode, name):
+    inp = wl.make_decode(5, 3, 128, 0, 0, seqlens=[1, 33, 512, 513, 1300], seed=6, device="cuda")
+    y = run_decode(inp, mode)
+    want = oracle_decode(inp, [(s, h) for s in range(5) for h in range(3)], name)
     got = np.stack([wl.to_f64(y[s, h]) for (s, h) in want])
     assert_close(got, np.stack(list(want.values())))
 

@@ -9,8 +9,10 @@
 // ever written to memory.
 //
 // Work decomposition
-//   A cluster of two CTAs owns one 128-row query tile of one (batch, head).
-//   CTA rank i computes map i+1 only: S_i = Q_i K_i^T on the tensor cores,
+//   Persistent clusters of two CTAs.  An item is one 128-row query tile of one
+//   (batch, head); the items are ordered longest first (causal: the last
+//   query tiles) and dealt to the clusters in a snake.  Per item, CTA rank i
+//   computes map i+1 only: S_i = Q_i K_i^T on the tensor cores,
 //   its own online softmax (running max m_i and sum l_i per row), and
 //   O_i += P_i V.  Both CTAs stream the same V tiles.  Tensor memory per CTA
 //   (512 columns): S (fp32, one buffer) in columns [0, 128), P (bf16, two
@@ -23,6 +25,11 @@
 //   into the partner's shared memory, the partial sums of squares of each
 //   row are swapped, and each CTA stages its columns of
 //   (1 - lambda_init) * w * O / rms as bf16 and writes them with TMA stores.
+//   The two CTAs meet through mbarriers only (each side says when its
+//   receive buffer is free, the copies complete on the receiver's barrier,
+//   the sums of squares are released with a cluster-scope arrive), so the
+//   producer and MMA threads run on into the next item: its Q and K tiles
+//   load and its first S product runs while the epilogue finishes.
 //
 // Warp roles (256 threads)
 //   warp 0: TMA producer for Q_i and K_i      warp 2: TMA producer for V
@@ -82,7 +89,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + 2 * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + 2 * V_BYTES;
-  static constexpr int SMEM_USED = OFF_BAR + 256;
+  static constexpr int OFF_SSX = OFF_BAR + 256;  // float[128]: the partner's sums of squares
+  static constexpr int SMEM_USED = OFF_SSX + 512;
   static constexpr int EXCH_BYTES = kBM * HALF * 4;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
   static constexpr uint32_t TM_S = 0;            // S (fp32, 128 columns)
@@ -90,18 +98,22 @@ struct Cfg {
   static constexpr uint32_t TM_O = 256;
   static constexpr uint32_t TM_COLS = 512;
   static_assert(EXCH_BYTES <= V_BYTES, "exchange buffers must fit in one V stage each");
-  static_assert(kBM * HALF * 2 <= 2 * K_BYTES, "output staging must fit in the K stages");
+  static_assert(kBM * HALF * 2 <= V_BYTES, "output staging must fit in one V stage");
+  static_assert(SMEM_USED + 1024 <= 232448, "shared memory per CTA");
 
 };
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;  // per item; q_empty: the item's last S product has read Q
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full, s_free;
   uint64_t p_full[2], p_empty[2];
   uint64_t mma_done;
-  uint64_t exch_full;  // the partner's half of the output has landed
+  uint64_t exch_full;   // per item: the partner's half of the output has landed here
+  uint64_t peer_ready;  // per item: the partner's receive buffer is free (remote arrive)
+  uint64_t ss_full;     // per item: the partner's sums of squares are here (remote arrive)
+  uint64_t epi_free;    // per item: the epilogue is done with the V stages
   uint32_t tmem_base;
   int abort;
 };
@@ -110,7 +122,8 @@ struct Bars {
 
 struct PrefillParams {
   __nv_bfloat16* o;
-  int N, H, causal, n_qtiles;
+  int N, H, B, causal, n_qtiles;
+  int n_items;  // B * H * n_qtiles
   const float* lambda;
   const float* q_scale;  // QK8 only: float32 [B][H][2], one scale per (batch, head, map)
   const float* k_scale;
@@ -143,17 +156,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  float* ssx = reinterpret_cast<float*>(smem + C::OFF_SSX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();  // 0: map 1, 1: map 2
-  const int qtile = p.n_qtiles - 1 - static_cast<int>(blockIdx.x >> 1);  // heaviest tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const uint32_t partner = rank ^ 1u;
+  const int cid = static_cast<int>(blockIdx.x >> 1), n_clusters = static_cast<int>(gridDim.x >> 1);
   const int N = p.N;
   const int n_kvtiles = (N + kBN - 1) / kBN;
-  const int n_kv = p.causal ? min(qtile + 1, n_kvtiles) : n_kvtiles;
+  const int BH = p.B * p.H;
+
+  // This cluster's k-th item (-1 past the end): longest first, dealt in a snake.
+  auto item_of = [&](int k) -> int {
+    const int pos = (k & 1) ? (n_clusters - 1 - cid) : cid;
+    const long long i = static_cast<long long>(k) * n_clusters + pos;
+    return i < p.n_items ? static_cast<int>(i) : -1;
+  };
+  struct Item {
+    int qtile, h, b, n_kv;
+  };
+  auto decode = [&](int i) -> Item {
+    Item it;
+    it.qtile = p.n_qtiles - 1 - i / BH;
+    const int bh = i % BH;
+    it.b = bh / p.H;
+    it.h = bh % p.H;
+    it.n_kv = p.causal ? min(it.qtile + 1, n_kvtiles) : n_kvtiles;
+    return it;
+  };
 
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
@@ -166,9 +200,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->s_free, 4);
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->exch_full, 1);
+    mbar_init(&bars->peer_ready, 1);
+    mbar_init(&bars->ss_full, 1);
+    mbar_init(&bars->epi_free, 1);
     bars->abort = 0;
     fence_mbarrier_init();
-    mbar_arrive_expect_tx(&bars->exch_full, C::EXCH_BYTES);  // armed long before the partner sends
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tq);
@@ -182,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
@@ -193,43 +230,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------- Q / K producer --
     if (lane == 0) {
-      const int c1 = 2 * h + static_cast<int>(rank);
-      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-#pragma unroll
-      for (int blk = 0; blk < C::QBLK; ++blk)
-        tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * C::QBOX, c1, qtile * kBM, b);
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&bars->k_empty[st], ph ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
+      int gk = 0;  // K tiles issued (all items)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        const int c1 = 2 * it.h + static_cast<int>(rank);
+        // Q of this item replaces the last one's once that item's S products have read it
+        if (k > 0 && !(ok = mbar_wait(&bars->q_empty, (k - 1) & 1, wc))) break;
+        mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
 #pragma unroll
         for (int blk = 0; blk < C::QBLK; ++blk)
-          tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * C::QBOX, c1,
-                      j * kBN, b);
-        issued = j + 1;
+          tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * C::QBOX, c1, it.qtile * kBM, it.b);
+        for (int j = 0; j < it.n_kv; ++j, ++gk) {
+          const int st = gk & 1;
+          if (!(ok = mbar_wait(&bars->k_empty[st], ((gk >> 1) & 1) ^ 1, wc))) break;
+          mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
+#pragma unroll
+          for (int blk = 0; blk < C::QBLK; ++blk)
+            tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * C::QBOX, c1,
+                        j * kBN, it.b);
+        }
       }
-      // make sure nothing is still landing in shared memory before the epilogue reuses it
-      mbar_wait(&bars->q_full, 0, wdrain);
-      for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, wdrain);
+      // nothing may still be landing in shared memory when the CTA exits
+      for (int j = max(0, gk - 2); j < gk; ++j) mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, wdrain);
     }
     __syncwarp();
   } else if (warp == 2) {
     // -------------------------------------------------------- V producer --
     if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&bars->v_empty[st], ph ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
+      int gv = 0;  // V tiles issued (all items)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        // the previous item's epilogue uses both V stages for its exchange
+        if (k > 0 && !(ok = mbar_wait(&bars->epi_free, (k - 1) & 1, wc))) break;
+        for (int j = 0; j < it.n_kv; ++j, ++gv) {
+          const int st = gv & 1;
+          if (!(ok = mbar_wait(&bars->v_empty[st], ((gv >> 1) & 1) ^ 1, wc))) break;
+          mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
 #pragma unroll
-        for (int blk = 0; blk < C::VBLK; ++blk)
-          tma_load_4d(sV + st * C::V_BYTES + blk * C::BLK_BYTES, &tv, &bars->v_full[st], blk * 64, h, j * kBN, b);
-        issued = j + 1;
+          for (int blk = 0; blk < C::VBLK; ++blk)
+            tma_load_4d(sV + st * C::V_BYTES + blk * C::BLK_BYTES, &tv, &bars->v_full[st], blk * 64, it.h,
+                        j * kBN, it.b);
+        }
       }
-      for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, wdrain);
+      for (int j = max(0, gv - 2); j < gv; ++j) mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, wdrain);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -238,10 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = QK8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      // O += P_t V_t, with P from buffer t % 2 and V from stage t % 2
-      auto issue_pv = [&](int t) -> bool {
-        const int bb = t & 1;
-        const uint32_t ph = (t >> 1) & 1;
+      int gs = 0;  // S products issued (all items)
+      int gp = 0;  // PV products issued (all items)
+      // O (+)= P V for the next tile, with P from buffer gp % 2 and V from stage gp % 2;
+      // `first` starts a new item's O
+      auto issue_pv = [&](bool first) -> bool {
+        const int bb = gp & 1;
+        const uint32_t ph = (gp >> 1) & 1;
         if (!mbar_wait(&bars->v_full[bb], ph, wc)) return false;
         if (!mbar_wait(&bars->p_full[bb], ph, wc)) return false;
         tc_fence_after();
@@ -249,35 +301,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint32_t a_tmem = tmem + C::TM_P + 64 * bb + 8 * kk;
           const uint64_t bd = smem_desc_sw128(sVa + bb * C::V_BYTES + kk * 2048, C::BLK_BYTES, 1024);
-          umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->v_empty[bb]);
         umma_commit(&bars->p_empty[bb]);
+        ++gp;
         return true;
       };
-      bool ok = mbar_wait(&bars->q_full, 0, wc);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j & 1;
-        // S_j overwrites S_{j-1}: every softmax warp must have read it
-        if (j > 0 && !(ok = mbar_wait(&bars->s_free, (j - 1) & 1, wc))) break;
-        if (!(ok = mbar_wait(&bars->k_full[st], (j >> 1) & 1, wc))) break;
-        tc_fence_after();
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        if (!(ok = mbar_wait(&bars->q_full, k & 1, wc))) break;
+        for (int j = 0; ok && j < it.n_kv; ++j, ++gs) {
+          const int st = gs & 1;
+          // S overwrites the previous S tile: every softmax warp must have read it
+          if (gs > 0 && !(ok = mbar_wait(&bars->s_free, (gs - 1) & 1, wc))) break;
+          if (!(ok = mbar_wait(&bars->k_full[st], (gs >> 1) & 1, wc))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / C::KSTEP; ++kk) {  // each instruction takes 32 bytes of every row
-          const int blk = kk >> 2;
-          const uint32_t koff = (kk & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + koff, 16, 1024);
-          if constexpr (QK8)
-            umma_ss_f8(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-          else
-            umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / C::KSTEP; ++kk) {  // each instruction takes 32 bytes of every row
+            const int blk = kk >> 2;
+            const uint32_t koff = (kk & 3) * 32;
+            const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + koff, 16, 1024);
+            if constexpr (QK8)
+              umma_ss_f8(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            else
+              umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->k_empty[st]);
+          umma_commit(&bars->s_full);
+          if (j == it.n_kv - 1) umma_commit(&bars->q_empty);  // the item's S products are all issued
+          if (j > 0) ok = issue_pv(j == 1);
         }
-        umma_commit(&bars->k_empty[st]);
-        umma_commit(&bars->s_full);
-        if (j > 0) ok = issue_pv(j - 1);
+        if (ok) ok = issue_pv(it.n_kv == 1);
       }
-      if (ok) issue_pv(n_kv - 1);
       // drain: every issued MMA has completed before tensor memory is read or freed
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, wdrain);
@@ -285,227 +345,242 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
 
-  // ------------------------------------------------------------ softmax --
-  const bool is_sm = warp >= 4;
-  const int quarter = warp & 3;
-  const int r = quarter * 32 + lane;  // query row within the tile (= TMEM lane)
-  const int qrow = qtile * kBM + r;
-  const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-  float m_run = -INFINITY, l_run = 0.f;
-  bool sm_ok = true;
-  if (is_sm) {
-    float sc = kLog2e * rsqrtf(static_cast<float>(D));
-    if constexpr (QK8) {  // scores of the codes times the two groups' scales
-      const int g = (b * p.H + h) * 2 + static_cast<int>(rank);
-      sc *= __ldg(p.q_scale + g) * __ldg(p.k_scale + g);
-    }
-    // O and l *= alpha (the whole warp takes part; alpha = 1 leaves a row as it is)
-    auto rescale_o = [&](float alpha) {
-#pragma unroll
-      for (int c = 0; c < C::DV / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32_sync(tl + C::TM_O + 32 * c, ov);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-        tmem_st32(tl + C::TM_O + 32 * c, ov);
+  if (warp >= 4) {
+    // ------------------------------------------------ softmax + epilogue --
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row within the tile (= TMEM lane)
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float coef2 = map2_coefficient(p.mode, *p.lambda);  // c in softmax(S1) + c softmax(S2)
+    constexpr int HALF = C::HALF;
+    constexpr int NC = HALF / 4;  // float4 chunks per exchanged row
+    float* recv = reinterpret_cast<float*>(sV);              // V stage 0: the partner's half
+    float* stage = reinterpret_cast<float*>(sV + C::V_BYTES);  // V stage 1: the half sent, then the output
+    const uint32_t own0 = (rank == 0) ? 0 : HALF;   // columns this CTA finishes
+    const uint32_t send0 = (rank == 0) ? HALF : 0;  // columns it hands to the partner
+    int g = 0;  // S / P tiles consumed (all items)
+    bool sm_ok = true;
+    for (int k = 0;; ++k) {
+      const int idx = item_of(k);
+      if (idx < 0) break;
+      const Item it = decode(idx);
+      const int N_kv = it.n_kv;
+      const int qtile = it.qtile;
+      const int qrow = qtile * kBM + r;
+      float sc = kLog2e * rsqrtf(static_cast<float>(D));
+      if constexpr (QK8) {  // scores of the codes times the two groups' scales
+        const int gi = (it.b * p.H + it.h) * 2 + static_cast<int>(rank);
+        sc *= __ldg(p.q_scale + gi) * __ldg(p.k_scale + gi);
       }
-      tmem_st_wait();
-      l_run *= alpha;
-    };
-    for (int j = 0; j < n_kv; ++j) {
-      const int bb = j & 1;
-      if (!(sm_ok = mbar_wait(&bars->s_full, j & 1, wc))) break;
-      // S_j has completed, and with it every MMA issued before it, PV_{j-2}
-      // included: P buffer b is free.
-      tc_fence_after();
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tl + C::TM_S + 0, s0);
-      tmem_ld32(tl + C::TM_S + 32, s1);
-      tmem_ld32(tl + C::TM_S + 64, s2);
-      tmem_ld32(tl + C::TM_S + 96, s3);
-      tmem_ld_wait4(s0, s1, s2, s3);
-      // S is in registers: the next S tile may overwrite the buffer
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free);
-      float x[128];
+      float m_run = -INFINITY, l_run = 0.f;
+      // O and l *= alpha (the whole warp takes part; alpha = 1 leaves a row as it is)
+      auto rescale_o = [&](float alpha) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        x[i] = __uint_as_float(s0[i]);
-        x[32 + i] = __uint_as_float(s1[i]);
-        x[64 + i] = __uint_as_float(s2[i]);
-        x[96 + i] = __uint_as_float(s3[i]);
-      }
-      const int key0 = j * kBN;
-      if (key0 + kBN > N || (p.causal && j == qtile)) {
-        const int lim = (p.causal ? min(N - 1, qrow) : N - 1) - key0;  // last visible key of the tile
+        for (int c = 0; c < C::DV / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32_sync(tl + C::TM_O + 32 * c, ov);
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > lim) x[i] = -INFINITY;
-      }
-      if (j == 0) {  // the first tile sets the reference maximum
-        float mk[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mk[c] = x[c];
-#pragma unroll
-        for (int i = 8; i < 128; i += 8) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) mk[c] = fmaxf(mk[c], x[i + c]);
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tl + C::TM_O + 32 * c, ov);
         }
-        m_run = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])), fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7]))) * sc;
-      }
-      // P = exp2(s*c - m_run) into P[b], taken relative to the reference
-      // maximum m_run as it stands; the tile's own maximum is formed alongside.
-      float lsum = 0.f, t_mx = -INFINITY;
-      auto make_p = [&](bool with_max) {
-        const float mneg = -m_run;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        float mk[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mk[c] = -INFINITY;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a0 = x[64 * half + 2 * i], a1 = x[64 * half + 2 * i + 1];
-            if (with_max) mk[i & 7] = fmaxf(mk[i & 7], fmaxf(a0, a1));
-            const float p0 = fast_exp2(fmaf(a0, sc, mneg));
-            const float p1 = fast_exp2(fmaf(a1, sc, mneg));
-            acc[i & 3] += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(tl + C::TM_P + 64 * bb + 32 * half, pk);
-        }
-        lsum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        if (with_max)
-          t_mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])), fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7]))) * sc;
-      };
-      make_p(true);
-      // A jump of the maximum by more than 2^64 would overflow P: rescale O
-      // to the new maximum (after PV_{j-1} has completed) and redo P.
-      const bool hard = t_mx > m_run + kOverflowGuard;
-      if (__any_sync(0xffffffffu, hard)) {
         tmem_st_wait();
-        if (!(sm_ok = mbar_wait(&bars->p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wc))) break;
+        l_run *= alpha;
+      };
+      for (int j = 0; sm_ok && j < N_kv; ++j, ++g) {
+        const int bb = g & 1;
+        if (!(sm_ok = mbar_wait(&bars->s_full, g & 1, wc))) break;
+        // S_g has completed, and with it every MMA issued before it, PV_{g-2}
+        // included: P buffer b is free.
         tc_fence_after();
-        rescale_o(hard ? fast_exp2(m_run - t_mx) : 1.0f);
-        if (hard) m_run = t_mx;
-        make_p(false);
+        uint32_t s0[32], s1[32], s2[32], s3[32];
+        tmem_ld32(tl + C::TM_S + 0, s0);
+        tmem_ld32(tl + C::TM_S + 32, s1);
+        tmem_ld32(tl + C::TM_S + 64, s2);
+        tmem_ld32(tl + C::TM_S + 96, s3);
+        tmem_ld_wait4(s0, s1, s2, s3);
+        // S is in registers: the next S tile may overwrite the buffer
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+        float x[128];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(s0[i]);
+          x[32 + i] = __uint_as_float(s1[i]);
+          x[64 + i] = __uint_as_float(s2[i]);
+          x[96 + i] = __uint_as_float(s3[i]);
+        }
+        const int key0 = j * kBN;
+        if (key0 + kBN > N || (p.causal && j == qtile)) {
+          const int lim = (p.causal ? min(N - 1, qrow) : N - 1) - key0;  // last visible key of the tile
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i > lim) x[i] = -INFINITY;
+        }
+        if (j == 0) {  // the first tile sets the reference maximum
+          float mk[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mk[c] = x[c];
+#pragma unroll
+          for (int i = 8; i < 128; i += 8) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mk[c] = fmaxf(mk[c], x[i + c]);
+          }
+          m_run = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])), fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7]))) * sc;
+        }
+        // P = exp2(s*c - m_run) into P[b], taken relative to the reference
+        // maximum m_run as it stands; the tile's own maximum is formed alongside.
+        float lsum = 0.f, t_mx = -INFINITY;
+        auto make_p = [&](bool with_max) {
+          const float mneg = -m_run;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          float mk[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mk[c] = -INFINITY;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float a0 = x[64 * half + 2 * i], a1 = x[64 * half + 2 * i + 1];
+              if (with_max) mk[i & 7] = fmaxf(mk[i & 7], fmaxf(a0, a1));
+              const float p0 = fast_exp2(fmaf(a0, sc, mneg));
+              const float p1 = fast_exp2(fmaf(a1, sc, mneg));
+              acc[i & 3] += p0 + p1;
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st32(tl + C::TM_P + 64 * bb + 32 * half, pk);
+          }
+          lsum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          if (with_max)
+            t_mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])), fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7]))) * sc;
+        };
+        make_p(true);
+        // A jump of the maximum by more than 2^64 would overflow P: rescale O
+        // to the new maximum (after the previous tile's PV has completed) and redo P.
+        const bool hard = t_mx > m_run + kOverflowGuard;
+        if (__any_sync(0xffffffffu, hard)) {
+          tmem_st_wait();
+          if (!(sm_ok = mbar_wait(&bars->p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, wc))) break;
+          tc_fence_after();
+          rescale_o(hard ? fast_exp2(m_run - t_mx) : 1.0f);
+          if (hard) m_run = t_mx;
+          make_p(false);
+        }
+        tmem_st_wait();
+        l_run += lsum;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[bb]);
+        // Lazy rescale: keep the reference within 2^8 of the running maximum.
+        // O is rescaled once this tile's PV (which used the old reference) has completed.
+        const bool need = t_mx > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          if (!(sm_ok = mbar_wait(&bars->p_empty[bb], (g >> 1) & 1, wc))) break;
+          tc_fence_after();
+          rescale_o(need ? fast_exp2(m_run - t_mx) : 1.0f);
+          if (need) m_run = t_mx;
+        }
       }
-      tmem_st_wait();
-      l_run += lsum;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[bb]);
-      // Lazy rescale: keep the reference within 2^8 of the running maximum.
-      // O is rescaled once PV_j (which used the old reference) has completed.
-      const bool need = t_mx > m_run + kRescaleThreshold;
-      if (__any_sync(0xffffffffu, need)) {
-        if (!(sm_ok = mbar_wait(&bars->p_empty[bb], (j >> 1) & 1, wc))) break;
-        tc_fence_after();
-        rescale_o(need ? fast_exp2(m_run - t_mx) : 1.0f);
-        if (need) m_run = t_mx;
-      }
-    }
-    // O is complete once the last PV (and with it every earlier MMA) has
-    if (sm_ok) sm_ok = mbar_wait(&bars->p_empty[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, wc);
-    tc_fence_after();
-  }
+      // the loop above may stop early after an abort: keep the tile count in step
+      g = 0;
+      for (int kk = 0; kk <= k; ++kk) g += decode(item_of(kk)).n_kv;
 
-  // ----------------------------------------------------------- epilogue --
-  // After the first cluster barrier every MMA and TMA load of both CTAs has
-  // completed, so Q, K and V space is reused: sums of squares in the Q tile,
-  // the partner's half in V stage 0, the half sent to it in V stage 1, the
-  // bf16 output tile in the K stages.
-  float* ssx = reinterpret_cast<float*>(sQ);  // [128] the partner's sums of squares, written remotely
-  float* recv = reinterpret_cast<float*>(sV);
-  float* stage = reinterpret_cast<float*>(sV + C::V_BYTES);
-  uint8_t* sOut = sK;
-  const uint32_t partner = rank ^ 1u;
-  constexpr int HALF = C::HALF;
-  constexpr int NC = HALF / 4;  // float4 chunks per exchanged row
-  cluster_sync_all();  // both CTAs: main loops drained, buffers free
-  const float coef2 = map2_coefficient(p.mode, *p.lambda);  // c in softmax(S1) + c softmax(S2)
-  const int own0 = (rank == 0) ? 0 : HALF;   // columns this CTA finishes
-  const int send0 = (rank == 0) ? HALF : 0;  // columns it hands to the partner
-  float y[HALF];
-  float ss = 0.f;
-  if (is_sm) {
-    const float inv = (rank == 0) ? 1.0f / l_run : coef2 / l_run;
-    float* srow = stage + r * HALF;
-#pragma unroll
-    for (int c = 0; c < HALF / 32; ++c) {
-      uint32_t ov[32];
-      tmem_ld32_sync(tl + C::TM_O + send0 + 32 * c, ov);
-#pragma unroll
-      for (int f = 0; f < 8; ++f) {
-        const int chunk = (c * 8 + f) ^ (r % NC);
-        *reinterpret_cast<float4*>(srow + chunk * 4) =
-            make_float4(__uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
-                        __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
+      // ------------------------------------------------------ epilogue --
+      // O is complete once the item's last PV (and with it every earlier MMA) has.
+      if (sm_ok) sm_ok = mbar_wait(&bars->p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, wc);
+      tc_fence_after();
+      // Both V stages are free of this item's PV products: announce that this
+      // CTA's receive buffer is ready, with the exchange barrier armed first.
+      named_bar_sync(1, 128);
+      if (tid == 128) {
+        mbar_arrive_expect_tx(&bars->exch_full, C::EXCH_BYTES);
+        mbar_arrive_remote(map_to_cta(smem_u32(&bars->peer_ready), partner));
       }
-    }
-    fence_proxy_async_smem();  // the staged rows are read by the bulk copy (async proxy)
-    __syncwarp();
-    if (lane == 0) {
-      const int off = quarter * 32 * HALF;  // this warp's 32 rows, contiguous
-      bulk_copy_s2cluster(map_to_cta(smem_u32(recv + off), partner), stage + off, 32 * HALF * 4,
-                          map_to_cta(smem_u32(&bars->exch_full), partner));
-      bulk_commit_group();
-    }
-    mbar_wait(&bars->exch_full, 0, wdrain);  // the partner's half has landed
-    const float* rrow = recv + r * HALF;
+      const float inv = (rank == 0) ? 1.0f / l_run : coef2 / l_run;
+      float* srow = stage + r * HALF;
 #pragma unroll
-    for (int c = 0; c < HALF / 32; ++c) {
-      uint32_t ov[32];
-      tmem_ld32_sync(tl + C::TM_O + own0 + 32 * c, ov);
+      for (int c = 0; c < HALF / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32_sync(tl + C::TM_O + send0 + 32 * c, ov);
 #pragma unroll
-      for (int f = 0; f < 8; ++f) {
-        const int chunk = (c * 8 + f) ^ (r % NC);
-        const float4 xr = *reinterpret_cast<const float4*>(rrow + chunk * 4);
-        const float xs[4] = {xr.x, xr.y, xr.z, xr.w};
+        for (int f = 0; f < 8; ++f) {
+          const int chunk = (c * 8 + f) ^ (r % NC);
+          *reinterpret_cast<float4*>(srow + chunk * 4) =
+              make_float4(__uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                          __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
+        }
+      }
+      fence_proxy_async_smem();  // the staged rows are read by the bulk copy (async proxy)
+      __syncwarp();
+      // the partner's receive buffer must be free before this CTA writes into it
+      const bool peer_ok = mbar_wait_acq_cluster(&bars->peer_ready, k & 1, wc);
+      if (lane == 0 && peer_ok) {
+        const int off = quarter * 32 * HALF;  // this warp's 32 rows, contiguous
+        bulk_copy_s2cluster(map_to_cta(smem_u32(recv + off), partner), stage + off, 32 * HALF * 4,
+                            map_to_cta(smem_u32(&bars->exch_full), partner));
+        bulk_commit_group();
+      }
+      mbar_wait(&bars->exch_full, k & 1, wdrain);  // the partner's half has landed (even after an abort)
+      float y[HALF];
+      float ss = 0.f;
+      const float* rrow = recv + r * HALF;
+#pragma unroll
+      for (int c = 0; c < HALF / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32_sync(tl + C::TM_O + own0 + 32 * c, ov);
+#pragma unroll
+        for (int f = 0; f < 8; ++f) {
+          const int chunk = (c * 8 + f) ^ (r % NC);
+          const float4 xr = *reinterpret_cast<const float4*>(rrow + chunk * 4);
+          const float xs[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float val = fmaf(__uint_as_float(ov[4 * f + e]), inv, xs[e]);
+            y[32 * c + 4 * f + e] = val;
+            ss = fmaf(val, val, ss);
+          }
+        }
+      }
+      // this row's half of the sum of squares to the partner, released at cluster scope
+      st_cluster_f32(map_to_cta(smem_u32(ssx + r), partner), ss);
+      fence_acq_rel_cluster();
+      if (lane == 0 && peer_ok) bulk_wait_group_read0();  // the outgoing copy has left the staging rows
+      __syncwarp();
+      named_bar_sync(1, 128);
+      if (tid == 128) mbar_arrive_remote(map_to_cta(smem_u32(&bars->ss_full), partner));
+      mbar_wait_acq_cluster(&bars->ss_full, k & 1, wdrain);
+      const float rs = rsqrtf((ss + ssx[r]) / static_cast<float>(C::DV) + p.eps);
+      const float gsc = (1.0f - p.lambda_init) * rs;
+      // bf16 tile [64-column block][128 rows][64 columns], 128-byte swizzle, in the staging stage
+      const uint32_t sout = smem_u32(stage);
+#pragma unroll
+      for (int c8 = 0; c8 < HALF / 8; ++c8) {
+        uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float val = fmaf(__uint_as_float(ov[4 * f + e]), inv, xs[e]);
-          y[32 * c + 4 * f + e] = val;
-          ss = fmaf(val, val, ss);
+          const int c = 8 * c8 + 2 * e;
+          w4[e] = pack_bf16x2(y[c] * gsc * __ldg(p.rms_w + own0 + c), y[c + 1] * gsc * __ldg(p.rms_w + own0 + c + 1));
         }
+        const uint32_t a = sout + (c8 / 8) * C::BLK_BYTES + r * 128 + (((c8 % 8) ^ (r & 7)) << 4);
+        st_shared_v4(a, w4[0], w4[1], w4[2], w4[3]);
       }
-    }
-    st_cluster_f32(map_to_cta(smem_u32(ssx + r), partner), ss);
-    if (lane == 0) bulk_wait_group_read0();  // the outgoing copy has left this CTA's memory
-    __syncwarp();
-  }
-  cluster_sync_all();  // the partner's partial sums of squares visible; no remote access after this
-  if (is_sm) {
-    const float rs = rsqrtf((ss + ssx[r]) / static_cast<float>(C::DV) + p.eps);
-    const float gsc = (1.0f - p.lambda_init) * rs;
-    // bf16 tile [64-column block][128 rows][64 columns], 128-byte swizzle
+      fence_proxy_async_smem();  // the tile is read by the TMA store (async proxy)
+      named_bar_sync(1, 128);    // the four softmax warps have staged their rows
+      if (tid == 128) {
 #pragma unroll
-    for (int c8 = 0; c8 < HALF / 8; ++c8) {
-      uint32_t w4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = 8 * c8 + 2 * e;
-        w4[e] = pack_bf16x2(y[c] * gsc * __ldg(p.rms_w + own0 + c), y[c + 1] * gsc * __ldg(p.rms_w + own0 + c + 1));
+        for (int blk = 0; blk < HALF / 64; ++blk)
+          tma_store_4d(&to, stage + blk * (C::BLK_BYTES / 4), own0 + 64 * blk, it.h, qtile * kBM, it.b);  // rows >= N clipped
+        bulk_commit_group();
+        bulk_wait_group_read0();  // the staging stage must stay valid until the store has read it
+        mbar_arrive(&bars->epi_free);  // both V stages are free for the next item's V tiles
       }
-      const uint32_t a = smem_u32(sOut) + (c8 / 8) * C::BLK_BYTES + r * 128 + (((c8 % 8) ^ (r & 7)) << 4);
-      st_shared_v4(a, w4[0], w4[1], w4[2], w4[3]);
+      __syncwarp();
     }
-    fence_proxy_async_smem();  // the tile is read by the TMA store (async proxy)
-    named_bar_sync(1, 128);    // the four softmax warps have staged their rows
-    if (warp == 4 && lane == 0) {
-#pragma unroll
-      for (int blk = 0; blk < HALF / 64; ++blk)
-        tma_store_4d(&to, sOut + blk * C::BLK_BYTES, own0 + 64 * blk, h, qtile * kBM, b);  // rows >= N are clipped
-      bulk_commit_group();
-      bulk_wait_group_read0();  // shared memory must stay valid until the store has read it
-    }
-    __syncwarp();
   }
+
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no remote access to either CTA remains
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
@@ -514,13 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool QK8>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& to, const PrefillParams& prm, int B, cudaStream_t stream) {
+                            const CUtensorMap& to, const PrefillParams& prm, cudaStream_t stream) {
   using C = Cfg<D, QK8>;
   cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * prm.n_qtiles, prm.H, B);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_ALLOC;
   cfg.stream = stream;
@@ -531,6 +605,19 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // persistent grid: as many clusters as can be resident at once (looked up once per device)
+  static int max_clusters[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int& mc = max_clusters[dev];
+  if (mc == 0) {
+    cfg.gridDim = dim3(2 * 128, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QK8>, &cfg) != cudaSuccess || n < 1) n = 1;
+    mc = n;
+  }
+  const int clusters = prm.n_items < mc ? prm.n_items : mc;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
   return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8>, tq, tk, tv, to, prm);
 }
 
@@ -543,8 +630,10 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.N = N;
   prm.H = H;
+  prm.B = B;
   prm.causal = causal ? 1 : 0;
   prm.n_qtiles = (N + kBM - 1) / kBM;
+  prm.n_items = B * H * prm.n_qtiles;
   prm.lambda = lambda;
   prm.q_scale = q_scale;
   prm.k_scale = k_scale;
@@ -555,9 +644,9 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.status = ctl.status;
   prm.limit_ns = ctl.limit_ns;
   const bool qk8 = q_scale != nullptr;
-  if (qk8) return d == 128 ? launch_d<128, true>(tq, tk, tv, to, prm, B, stream) : cudaErrorInvalidValue;
-  if (d == 128) return launch_d<128, false>(tq, tk, tv, to, prm, B, stream);
-  if (d == 64) return launch_d<64, false>(tq, tk, tv, to, prm, B, stream);
+  if (qk8) return d == 128 ? launch_d<128, true>(tq, tk, tv, to, prm, stream) : cudaErrorInvalidValue;
+  if (d == 128) return launch_d<128, false>(tq, tk, tv, to, prm, stream);
+  if (d == 64) return launch_d<64, false>(tq, tk, tv, to, prm, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -10,8 +10,10 @@
 //
 // Work decomposition
 //   Persistent clusters of two CTAs.  An item is one 128-row query tile of one
-//   (batch, head); the items are ordered longest first (causal: the last
-//   query tiles) and dealt to the clusters in a snake.  Per item, CTA rank i
+//   (batch, head).  The (batch, head) pairs are taken in groups whose K and V
+//   fit in about 48 MB of L2 together; within a group the items are ordered
+//   longest first (causal: the last query tiles); the whole list is dealt to
+//   the clusters in a snake.  Per item, CTA rank i
 //   computes map i+1 only: S_i = Q_i K_i^T on the tensor cores,
 //   its own online softmax (running max m_i and sum l_i per row), and
 //   O_i += P_i V.  Both CTAs stream the same V tiles.  Tensor memory per CTA
@@ -123,7 +125,8 @@ struct Bars {
 struct PrefillParams {
   __nv_bfloat16* o;
   int N, H, B, causal, n_qtiles;
-  int n_items;  // B * H * n_qtiles
+  int n_items;     // B * H * n_qtiles
+  int head_group;  // (batch, head) pairs per item group (K and V of a group stay in L2)
   const float* lambda;
   const float* q_scale;  // QK8 only: float32 [B][H][2], one scale per (batch, head, map)
   const float* k_scale;
@@ -177,8 +180,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto decode = [&](int i) -> Item {
     Item it;
-    it.qtile = p.n_qtiles - 1 - i / BH;
-    const int bh = i % BH;
+    const int per_group = p.head_group * p.n_qtiles;
+    const int grp = i / per_group, li = i % per_group;
+    const int gsize = min(p.head_group, BH - grp * p.head_group);  // the last group may be smaller
+    it.qtile = p.n_qtiles - 1 - li / gsize;
+    const int bh = grp * p.head_group + li % gsize;
     it.b = bh / p.H;
     it.h = bh % p.H;
     it.n_kv = p.causal ? min(it.qtile + 1, n_kvtiles) : n_kvtiles;
@@ -634,6 +640,11 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.causal = causal ? 1 : 0;
   prm.n_qtiles = (N + kBM - 1) / kBM;
   prm.n_items = B * H * prm.n_qtiles;
+  {  // pairs per group: their K (both maps) and V, 8d bytes per token, in about 48 MB
+    const long long per_head = static_cast<long long>(N) * 8 * d;
+    const long long grp = (48ll << 20) / (per_head > 0 ? per_head : 1);
+    prm.head_group = static_cast<int>(grp < 1 ? 1 : (grp > B * H ? B * H : grp));
+  }
   prm.lambda = lambda;
   prm.q_scale = q_scale;
   prm.k_scale = k_scale;

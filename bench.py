@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-qk8", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
-    ap.add_argument("--bwd-steps", type=int, default=5)
+    ap.add_argument("--bwd-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
@@ -247,24 +247,27 @@ def cpu_baseline(inp, budget_s):
 # --------------------------------------------------------------- reference --
 
 # fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flops per FMA x 1965 MHz
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-
-
-def bench_bwd(api, inp, lam, reduce_max, barrier, K):
-    """The backward pass (training) on the same workload: dq, dk, dv, dlambda and
-    the norm weight's gradient for a seeded upstream gradient dy."""
+def bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, K):
+    """The backward pass (training) on the same workload, on the tensor cores
+    (diffattn_bwd_tc): dq, dk, dv, dlambda and the norm weight's gradient for a
+    seeded upstream gradient dy.  One step = the statistics pass (the prefill
+    recomputed for A_i V and the log-sum-exps), the per-row dO pass and the dV,
+    dK and dQ kernels."""
     import torch
 
     B, N, H, _, d = inp.q.shape
     g = torch.Generator(device=inp.q.device).manual_seed(4321)
     dy = torch.randn(inp.v.shape, generator=g, device=inp.q.device).to(inp.v.dtype)
-    ws = torch.empty(api.bwd_workspace_size(B, N, H, d), dtype=torch.uint8, device=inp.q.device)
+    ws = torch.empty(api.bwd_tc_workspace_size(B, N, H, d), dtype=torch.uint8, device=inp.q.device)
+    f32 = dict(dtype=torch.float32, device=inp.q.device)
+    outs = (torch.empty(inp.q.shape, **f32), torch.empty(inp.k.shape, **f32), torch.empty(inp.v.shape, **f32),
+            torch.empty(1, **f32), torch.empty(2 * d, **f32))
 
     def step():
-        return api.diffattn_bwd(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
-                                workspace=ws)
+        return api.diffattn_bwd_tc(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
+                                   workspace=ws, out=outs)
 
-    for _ in range(2):
+    for _ in range(3):
         step()
     torch.cuda.synchronize()
     barrier()
@@ -276,18 +279,26 @@ def bench_bwd(api, inp, lam, reduce_max, barrier, K):
     torch.cuda.synchronize()
     ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev))
     pairs = B * H * (N * (N + 1) // 2 if inp.causal else N * N)
-    # algorithmic: per visible (query, key) pair, 20 d flops -- recomputing both maps'
-    # scores (2 d MACs), dA = G V^T once (2 d), dV (2 d), dQ_i and dK_i (2 x 2 d)
+    # algorithmic: per visible (query, key) pair, 20 d flops -- both maps' scores
+    # (2 x 2d), dA = G V^T once (4d), dV (4d), dQ_i and dK_i (2 x 2 x 2d)
     alg = 20.0 * d * pairs
-    executed = 40.0 * d * pairs  # the row pass recomputes the forward; both gradient passes recompute S and dA
+    # executed: the statistics pass (12 d: scores 4d, both PV 8d), dV kernel
+    # (scores 4d + dV 4d), dK and dQ kernels (scores 4d + dP 4d + 4d each)
+    executed = 44.0 * d * pairs
+    loop_ms = ms * K
+    sustained = loop_ms >= 1000.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     achieved = alg / (ms * 1e-3) / 1e12
     return {"metric": "DiffAttn backward TFLOP/s (dq, dk, dv, dlambda, dw)", "value": achieved, "unit": "TFLOP/s",
             "steps": K, "ms_per_step": ms, "flops_per_step_algorithmic": alg, "flops_per_step_executed": executed,
-            "roofline": {"bound": "alu", "achieved": executed / (ms * 1e-3) / 1e12, "peak": FP32_ALU_TFLOPS,
-                         "unit": "TFLOP/s", "frac": executed / (ms * 1e-3) / 1e12 / FP32_ALU_TFLOPS,
-                         "traffic": None, "kernel": "bwd_rows + bwd_keys + bwd_queries (CUDA cores, fp32)",
-                         "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz"},
-            "gpu_launches": 3 * K}
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "executed_tflops": executed / (ms * 1e-3) / 1e12,
+                         "kernel": "prefill_sm100_kernel (statistics mode) + bwd_prep + bwd_grad_sm100 x3 (dV, dK, dQ)",
+                         "peak_source": f"{peak_src} bf16 dense, " + (
+                             f"sustained (timed loop {loop_ms / 1e3:.2f} s)" if sustained
+                             else f"burst (timed loop {loop_ms / 1e3:.2f} s)")},
+            "gpu_launches": 5 * K}
 
 
 def bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K):
@@ -521,7 +532,7 @@ def run_ours(args):
     }
 
     if not args.no_bwd:
-        line["bwd"] = bench_bwd(api, inp, lam, reduce_max, barrier, args.bwd_steps)
+        line["bwd"] = bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, args.bwd_steps)
     if not args.no_qk8 and d == 128:
         line["qk8"] = bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8))
     if not args.no_decode:

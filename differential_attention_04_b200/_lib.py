@@ -27,6 +27,9 @@ SIGNATURES = {
     "diffattn_bwd_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
                               _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "diffattn_bwd_tc_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "diffattn_bwd_tc": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
+                                 _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "diffattn_lambda_bwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "diffattn_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _c_float,

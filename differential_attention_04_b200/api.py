@@ -160,6 +160,35 @@ def diffattn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch.Te
     return dq, dk, dv, dlam, dw
 
 
+def bwd_tc_workspace_size(B: int, N: int, H: int, d: int) -> int:
+    return int(lib().diffattn_bwd_tc_workspace_size(B, N, H, d))
+
+
+def diffattn_bwd_tc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch.Tensor, lam: torch.Tensor,
+                    lambda_init: float, rms_w: torch.Tensor, eps: float = 1e-5, causal: bool = True,
+                    mode: int = MODE_DIFF, workspace: torch.Tensor | None = None, out=None):
+    """Tensor-core backward of the prefill: (dq, dk, dv, dlambda, drms_w), float32, for bfloat16 q, k, v and
+    upstream gradient dy (shaped like v), d = 64 or 128.  `out` may hold preallocated outputs in that order."""
+    _dev(q, k, v, dy, lam, rms_w)
+    B, N, H, two, d = q.shape
+    if two != 2 or k.shape != q.shape or tuple(v.shape) != (B, N, H, 2 * d) or dy.shape != v.shape:
+        raise ValueError("shapes must be q, k: [B, N, H, 2, d] and v, dy: [B, N, H, 2d]")
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, dy)):
+        raise ValueError("q, k, v, dy must be bfloat16")
+    if out is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        out = (torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32),
+               torch.empty(1, **f32), torch.empty(2 * d, **f32))
+    dq, dk, dv, dlam, dw = out
+    if workspace is None:
+        workspace = torch.empty(bwd_tc_workspace_size(B, N, H, d), dtype=torch.uint8, device=q.device)
+    _check("diffattn_bwd_tc", lib().diffattn_bwd_tc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dy), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+        _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream()))
+    return dq, dk, dv, dlam, dw
+
+
 def diffattn_lambda_bwd(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor, lk2: torch.Tensor,
                         dlam: torch.Tensor):
     """Gradients (dlq1, dlk1, dlq2, dlk2) of the lambda re-parameterisation for a device dlambda."""

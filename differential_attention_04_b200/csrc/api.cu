@@ -61,16 +61,16 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over a row-major tensor with dims (innermost first) d0..d3 of bf16
-// (esize 2) or byte (esize 1) elements; box = 128 bytes x 1 x 128 x 1,
+// (esize 2) or byte (esize 1) elements; box = 128 bytes x 1 x box_rows x 1,
 // 128-byte swizzle, zero fill out of bounds.
 bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
-               int esize = 2) {
+               int esize = 2, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const uint64_t e = static_cast<uint64_t>(esize);
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
   const cuuint64_t strides[3] = {d0 * e, d0 * d1 * e, d0 * d1 * d2 * e};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 1, 128, 1};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 1, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
             const_cast<void*>(base), dims, strides, box, estr,
@@ -221,6 +221,43 @@ int diffattn_bwd(const void* q, const void* k, const void* v, const void* dy, in
     return DIFFATTN_ERR_WORKSPACE;
   return cuda_status(launch_bwd(q, k, v, dy, dtype == DIFFATTN_BF16, B, N, H, d, causal, lambda, lambda_init,
                                 rms_w, eps, mode, dq, dk, dv, dlambda, drms_w, workspace, stream));
+}
+
+size_t diffattn_bwd_tc_workspace_size(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return 0;
+  return bwd_tc_layout(B, N, H, d).bytes;
+}
+
+int diffattn_bwd_tc(const void* q, const void* k, const void* v, const void* dy, int B, int N, int H, int d,
+                    int causal, const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                    float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
+                    size_t ws_bytes, cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !dy || !lambda || !rms_w || !dq || !dk || !dv || !dlambda || !drms_w)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * ((N + 127) / 128) > 0x7fffffffll) return DIFFATTN_ERR_UNSUPPORTED;
+  const BwdTcLayout L = bwd_tc_layout(B, N, H, d);
+  if (!workspace || ws_bytes < L.bytes || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
+  const void* g = static_cast<const char*>(workspace) + L.off_g;
+  BwdTcMaps m;
+  if (!encode_4d(&m.q128, q, d, 2ull * H, N, B) || !encode_4d(&m.q32, q, d, 2ull * H, N, B, 2, 32) ||
+      !encode_4d(&m.k128, k, d, 2ull * H, N, B) || !encode_4d(&m.k32, k, d, 2ull * H, N, B, 2, 32) ||
+      !encode_4d(&m.v128, v, 2ull * d, H, N, B) || !encode_4d(&m.v32, v, 2ull * d, H, N, B, 2, 32) ||
+      !encode_4d(&m.g128, g, 2ull * d, H, N, B) || !encode_4d(&m.g32, g, 2ull * d, H, N, B, 2, 32))
+    return DIFFATTN_ERR_CUDA;
+  DevCtl ctl;
+  if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  ctl.limit_ns = g_wait_limit_ns.load();
+  return cuda_status(launch_bwd_sm100(m, dy, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv,
+                                      dlambda, drms_w, workspace, ctl, stream));
 }
 
 int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,

@@ -47,6 +47,28 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
                        int d, int causal, const float* lambda, float lambda_init, const float* rms_w, float eps,
                        int mode, float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
                        cudaStream_t stream);
+// Tensor-core backward (bf16 inputs, d in {64, 128}).  Maps over q, k
+// [B, N, H*2, d] and v, G [B, N, H, 2d] with boxes of 128 bytes x 128 rows
+// (q128 ...) or x 32 rows (q32 ...); G is the workspace's bf16 dO.
+struct BwdTcMaps {
+  CUtensorMap q128, q32, k128, k32, v128, v32, g128, g32;
+};
+// Workspace: per map A_i V as float32 [B, N, H, 2, 2d]; G bf16 [B, N, H, 2d];
+// statistics float4 [B][H][n_pad] (n_pad = N rounded up to 128).
+struct BwdTcLayout {
+  size_t off_omaps, off_g, off_stats, bytes;
+  int n_pad;
+};
+BwdTcLayout bwd_tc_layout(int B, int N, int H, int d);
+cudaError_t launch_bwd_sm100(const BwdTcMaps& m, const void* dy, int B, int N, int H, int d, int causal,
+                             const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                             float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
+                             DevCtl ctl, cudaStream_t stream);
+// The tcgen05 prefill in its statistics mode: per map, O_i / l_i into
+// o_maps and the log2-sum-exp into component i of the float4 rows of lse.
+cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, int B,
+                                       int N, int H, int d, int causal, const float* lambda, float* o_maps,
+                                       float* lse, int n_pad, DevCtl ctl, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
                               const float* dlambda, float* dlq1, float* dlk1, float* dlq2, float* dlk2,
                               cudaStream_t stream);

@@ -136,6 +136,10 @@ struct PrefillParams {
   float eps;
   int* status;
   unsigned long long limit_ns;
+  // statistics mode (the backward pass's forward): per map, O_i / l_i and the log-sum-exp
+  float* o_maps;  // float32 [B, N, H, 2, 2d]
+  float* lse;     // float32 view of float4 [B][H][n_pad]: component i = map i's log2-sum-exp
+  int n_pad;
 };
 
 // Wait for every tcgen05.ld issued so far and pin 128 registers behind the wait.
@@ -147,7 +151,9 @@ __device__ __forceinline__ void tmem_ld_wait4(uint32_t (&a)[32], uint32_t (&b)[3
   tmem_ld_wait(d);
 }
 
-template <int D, bool QK8>
+// STATS: instead of the normalised output, each CTA writes its own map's
+// O_i / l_i (float32) and log-sum-exp, for the backward pass.
+template <int D, bool QK8, bool STATS>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                          const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -495,6 +501,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O is complete once the item's last PV (and with it every earlier MMA) has.
       if (sm_ok) sm_ok = mbar_wait(&bars->p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, wc);
       tc_fence_after();
+      if constexpr (STATS) {
+        // This map's O_i / l_i for the row, and lse_i = m + log2(l) in the
+        // scaled log2 units of P = exp2(s * sc - m): P / l = exp2(s * sc - lse_i).
+        const bool live = qrow < N;
+        const float inv = 1.0f / l_run;
+        float* orow = p.o_maps + ((static_cast<size_t>(it.b) * N + (live ? qrow : 0)) * p.H + it.h) * (2 * C::DV) +
+                      rank * C::DV;
+#pragma unroll 1
+        for (int c = 0; c < C::DV / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32_sync(tl + C::TM_O + 32 * c, ov);
+          if (live) {
+#pragma unroll
+            for (int f = 0; f < 8; ++f)
+              *reinterpret_cast<float4*>(orow + 32 * c + 4 * f) =
+                  make_float4(__uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                              __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
+          }
+        }
+        if (live) p.lse[((static_cast<size_t>(it.b) * p.H + it.h) * p.n_pad + qrow) * 4 + rank] = m_run + log2f(l_run);
+        tc_fence_before();
+        named_bar_sync(1, 128);  // every row's tensor-memory reads are done
+        if (tid == 128) mbar_arrive(&bars->epi_free);  // the next item's first PV may overwrite O
+        __syncwarp();
+        continue;
+      }
       // Both V stages are free of this item's PV products: announce that this
       // CTA's receive buffer is ready, with the exchange barrier armed first.
       named_bar_sync(1, 128);
@@ -593,11 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool QK8>
+template <int D, bool QK8, bool STATS = false>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const PrefillParams& prm, cudaStream_t stream) {
   using C = Cfg<D, QK8>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8, STATS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -619,12 +651,12 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if (mc == 0) {
     cfg.gridDim = dim3(2 * 128, 1, 1);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QK8>, &cfg) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QK8, STATS>, &cfg) != cudaSuccess || n < 1) n = 1;
     mc = n;
   }
   const int clusters = prm.n_items < mc ? prm.n_items : mc;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8>, tq, tk, tv, to, prm);
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8, STATS>, tq, tk, tv, to, prm);
 }
 
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -632,7 +664,7 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, int mode, const float* q_scale,
                                  const float* k_scale, DevCtl ctl, cudaStream_t stream) {
-  PrefillParams prm;
+  PrefillParams prm = {};
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.N = N;
   prm.H = H;
@@ -658,6 +690,36 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   if (qk8) return d == 128 ? launch_d<128, true>(tq, tk, tv, to, prm, stream) : cudaErrorInvalidValue;
   if (d == 128) return launch_d<128, false>(tq, tk, tv, to, prm, stream);
   if (d == 64) return launch_d<64, false>(tq, tk, tv, to, prm, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, int B,
+                                       int N, int H, int d, int causal, const float* lambda, float* o_maps,
+                                       float* lse, int n_pad, DevCtl ctl, cudaStream_t stream) {
+  PrefillParams prm = {};
+  prm.N = N;
+  prm.H = H;
+  prm.B = B;
+  prm.causal = causal ? 1 : 0;
+  prm.n_qtiles = (N + kBM - 1) / kBM;
+  prm.n_items = B * H * prm.n_qtiles;
+  {
+    const long long per_head = static_cast<long long>(N) * 8 * d;
+    const long long grp = (48ll << 20) / (per_head > 0 ? per_head : 1);
+    prm.head_group = static_cast<int>(grp < 1 ? 1 : (grp > B * H ? B * H : grp));
+  }
+  prm.lambda = lambda;
+  prm.mode = 0;
+  prm.lambda_init = 0.f;
+  prm.eps = 1.f;
+  prm.status = ctl.status;
+  prm.limit_ns = ctl.limit_ns;
+  prm.o_maps = o_maps;
+  prm.lse = lse;
+  prm.n_pad = n_pad;
+  // the output map is never used in this mode: tv stands in for it
+  if (d == 128) return launch_d<128, false, true>(tq, tk, tv, tv, prm, stream);
+  if (d == 64) return launch_d<64, false, true>(tq, tk, tv, tv, prm, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -3,6 +3,7 @@
   python -m differential_attention_04_b200.run_case prefill --B 2 --N 4096 --H 12 --d 128 --causal 1 --iters 3
   python -m differential_attention_04_b200.run_case prefill --qk8 1 ...   (e4m3 queries/keys: quantise + forward;
                                                                           2: forward only; 3: quantise only)
+  python -m differential_attention_04_b200.run_case bwd --tc 1 ...   (tensor-core backward; 0: CUDA cores)
   python -m differential_attention_04_b200.run_case decode --S 64 --H 12 --lmin 1024 --lmax 4096 --iters 3
 
 Inputs come from the seeded generators in ``workloads``; the output is not
@@ -29,6 +30,7 @@ def main(argv=None):
     ap.add_argument("--causal", type=int, default=1)
     ap.add_argument("--dtype", default="bf16")
     ap.add_argument("--qk8", type=int, default=0)
+    ap.add_argument("--tc", type=int, default=1)
     ap.add_argument("--S", type=int, default=64)
     ap.add_argument("--lmin", type=int, default=1024)
     ap.add_argument("--lmax", type=int, default=4096)
@@ -60,9 +62,14 @@ def main(argv=None):
         inp = wl.make_prefill(a.B, a.N, a.H, a.d, causal=bool(a.causal), dtype=a.dtype, seed=a.seed, device=dev)
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
         dy = torch.randn(inp.v.shape, device=dev).to(inp.v.dtype)
-        ws = torch.empty(api.bwd_workspace_size(a.B, a.N, a.H, a.d), dtype=torch.uint8, device=dev)
-        run = lambda: api.diffattn_bwd(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps,
-                                       inp.causal, workspace=ws)
+        if a.tc:
+            ws = torch.empty(api.bwd_tc_workspace_size(a.B, a.N, a.H, a.d), dtype=torch.uint8, device=dev)
+            run = lambda: api.diffattn_bwd_tc(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps,
+                                              inp.causal, workspace=ws)
+        else:
+            ws = torch.empty(api.bwd_workspace_size(a.B, a.N, a.H, a.d), dtype=torch.uint8, device=dev)
+            run = lambda: api.diffattn_bwd(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps,
+                                           inp.causal, workspace=ws)
     else:
         inp = wl.make_decode(a.S, a.H, a.d, a.lmin, a.lmax, seed=a.seed, device=dev)
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)

@@ -153,6 +153,39 @@ int diffattn_bwd(const void* q, const void* k, const void* v, const void* dy,
                  cudaStream_t stream);
 
 /*
+ * Tensor-core backward pass: the gradients diffattn_bwd defines, computed
+ * with tcgen05 products from bf16 operands, as a training step would.
+ * P, G = dO and dS are rounded to bf16 before each product (fp32
+ * accumulation), so the gradients carry bf16-level errors (normwise about
+ * 1e-3 relative) where diffattn_bwd carries fp32-level ones.
+ *
+ * diffattn_bwd_tc_workspace_size -- bytes of workspace for diffattn_bwd_tc
+ *   (0 for sizes below 1): fp32 [B, N, H, 2, 2d] (each map's A_i V), bf16
+ *   [B, N, H, 2d] (dO) and 16 bytes per (b, h, n) with n rounded up to 128.
+ * diffattn_bwd_tc
+ *   q, k        : device bf16 [B, N, H, 2, d], d = 64 or 128
+ *   v, dy       : device bf16 [B, N, H, 2d]
+ *   other arguments, outputs and layouts as in diffattn_bwd
+ *   workspace   : device, >= diffattn_bwd_tc_workspace_size bytes, 16-byte aligned
+ * Five stream-ordered launches: the prefill in a statistics mode (per map
+ * A_i V and the log-sum-exp per row), a per-row pass for dO, dw and dlambda,
+ * and one kernel each for dV, dK and dQ.  No allocation.  dlambda and drms_w
+ * are summed with atomics (last bits may vary from run to run); dq, dk, dv
+ * are deterministic.
+ * Errors: DIFFATTN_ERR_INVALID_ARG (null or unaligned pointers, bad mode or
+ * sizes), DIFFATTN_ERR_UNSUPPORTED (d other than 64 or 128),
+ * DIFFATTN_ERR_WORKSPACE, DIFFATTN_ERR_CUDA; DIFFATTN_ERR_TIMEOUT through
+ * diffattn_device_status if a kernel wait ran out.
+ */
+size_t diffattn_bwd_tc_workspace_size(int B, int N, int H, int d);
+int diffattn_bwd_tc(const void* q, const void* k, const void* v, const void* dy,
+                    int B, int N, int H, int d, int causal,
+                    const float* lambda, float lambda_init, const float* rms_w,
+                    float eps, int mode, float* dq, float* dk, float* dv,
+                    float* dlambda, float* drms_w, void* workspace, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/*
  * diffattn_lambda_bwd -- gradients of the lambda re-parameterisation (Eq. 2)
  * for a device dlambda: dlq1 = dlambda e1 lk1, dlk1 = dlambda e1 lq1,
  * dlq2 = -dlambda e2 lk2, dlk2 = -dlambda e2 lq2, with e1 = exp(lq1 . lk1),

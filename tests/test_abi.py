@@ -95,6 +95,24 @@ def test_validation_without_gpu(L):
     assert L.diffattn_bwd_workspace_size(1, 16, 2, 64) == 4 * 16 * 2 * 128 + 16 * 16 * 2
     assert L.diffattn_bwd_workspace_size(0, 16, 2, 64) == 0
     assert L.diffattn_lambda_bwd(nul, nul, nul, nul, 8, nul, nul, nul, nul, nul, nul) == api.ERR_INVALID_ARG
+    # tensor-core backward: d in {64, 128}, aligned pointers, enough workspace
+    tc = lambda x, N, d, ws, wsb, mode=0: L.diffattn_bwd_tc(x, x, x, x, 1, N, 2, d, 1, x, 0.5, x, 1e-5, mode,
+                                                            x, x, x, x, x, ws, wsb, nul)
+    assert tc(fake, 16, 96, fake, 1 << 30) == api.ERR_UNSUPPORTED
+    assert tc(fake, 16, 32, fake, 1 << 30) == api.ERR_UNSUPPORTED
+    assert tc(fake, 16, 128, nul, 1 << 30) == api.ERR_WORKSPACE
+    assert tc(fake, 16, 128, fake, 16) == api.ERR_WORKSPACE
+    assert tc(nul, 16, 128, fake, 1 << 30) == api.ERR_INVALID_ARG
+    assert tc(ctypes.c_void_p(4104), 16, 128, fake, 1 << 30) == api.ERR_INVALID_ARG
+    assert tc(fake, 16, 128, fake, 1 << 30, mode=4) == api.ERR_INVALID_ARG
+    assert tc(fake, 0, 128, fake, 1 << 30) == api.ERR_INVALID_ARG
+    # per map A_i V (float32), dO (bf16), 16 bytes per (b, h, n) with n rounded up to 128; 256-byte sections
+    up = lambda x: (x + 255) // 256 * 256
+    assert L.diffattn_bwd_tc_workspace_size(1, 16, 2, 64) == up(4 * 16 * 2 * 2 * 128) + up(2 * 16 * 2 * 128) + \
+        up(16 * 2 * 128)
+    assert L.diffattn_bwd_tc_workspace_size(2, 300, 3, 128) == up(4 * 600 * 3 * 2 * 256) + up(2 * 600 * 3 * 256) + \
+        up(16 * 2 * 3 * 384)
+    assert L.diffattn_bwd_tc_workspace_size(1, 0, 2, 64) == 0
     # decode
     dec = lambda q, d, ws, wsb, S=4: L.diffattn_decode(q, q, q, q, 100, q, S, 2, d, q, 0.5, q, 1e-5, ws, wsb, nul)
     assert dec(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG

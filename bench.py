@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-qk8", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--bwd-steps", type=int, default=50)
+    ap.add_argument("--no-proj", action="store_true")
+    ap.add_argument("--proj-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
@@ -301,6 +303,57 @@ def bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, K):
             "gpu_launches": 5 * K}
 
 
+def bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, K):
+    """The dense steps either side of the path at the 3B-like model's shapes
+    (B=4, N=4096, d_model=3072, H=12, d=128): the query/key/value projection
+    with the rotary embedding fused into its epilogue, then the output
+    projection of the heads' outputs.  One step = both GEMMs."""
+    import torch
+
+    inp = wl.make_proj_case("proj_3b", seed=0, device=dev)
+    B, N, H, d = inp.B, inp.N, inp.H, inp.d
+    dm = inp.x.shape[1]
+    table = api.rope_table(N, d)
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    qkv = (torch.empty((B, N, H, 2, d), **bf), torch.empty((B, N, H, 2, d), **bf), torch.empty((B, N, H, 2 * d), **bf))
+    y = torch.empty((B * N, dm), **bf)
+
+    def step():
+        api.qkv_proj(inp.x, inp.w_qkv, B, N, H, d, table, out=qkv)
+        api.out_proj(qkv[2], inp.w_o, out=y)  # V stands in for the attention output: same shape and dtype
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for e0, e1, e2 in ev:
+        e0.record()
+        api.qkv_proj(inp.x, inp.w_qkv, B, N, H, d, table, out=qkv)
+        e1.record()
+        api.out_proj(qkv[2], inp.w_o, out=y)
+        e2.record()
+    torch.cuda.synchronize()
+    q_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b, _ in ev))
+    o_ms = reduce_max(statistics.mean(b.elapsed_time(c) for _, b, c in ev))
+    M = B * N
+    f_qkv = 2.0 * M * dm * (3 * H * 2 * d)
+    f_o = 2.0 * M * (H * 2 * d) * dm
+    loop_ms = (q_ms + o_ms) * K
+    sustained = loop_ms >= 1000.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    achieved = (f_qkv + f_o) / ((q_ms + o_ms) * 1e-3) / 1e12
+    return {"metric": "QKV projection + RoPE and output projection TFLOP/s (3B-like shapes)", "value": achieved,
+            "unit": "TFLOP/s", "steps": K, "ms_per_step": q_ms + o_ms, "qkv_rope_ms": q_ms, "out_proj_ms": o_ms,
+            "qkv_tflops": f_qkv / (q_ms * 1e-3) / 1e12, "out_tflops": f_o / (o_ms * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "proj_gemm_sm100_kernel (x2)",
+                         "peak_source": f"{peak_src} bf16 dense, " + (
+                             f"sustained (timed loop {loop_ms / 1e3:.2f} s)" if sustained
+                             else f"burst (timed loop {loop_ms / 1e3:.2f} s)")},
+            "gpu_launches": 2 * K}
+
+
 def bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K):
     """The e4m3 query/key variant on the same workload: a step quantises q and k
     (one absmax scale per batch, head and map) and runs the prefill whose
@@ -533,6 +586,8 @@ def run_ours(args):
 
     if not args.no_bwd:
         line["bwd"] = bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, args.bwd_steps)
+    if not args.no_proj:
+        line["proj"] = bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, args.proj_steps)
     if not args.no_qk8 and d == 128:
         line["qk8"] = bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8))
     if not args.no_decode:

@@ -30,6 +30,9 @@ SIGNATURES = {
     "diffattn_bwd_tc_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_bwd_tc": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
                                  _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "diffattn_rope_table": (_c_int, [_c_int, _c_int, ctypes.c_double, _vp, _vp]),
+    "diffattn_qkv_proj": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
+    "diffattn_out_proj": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp]),
     "diffattn_lambda_bwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "diffattn_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _c_float,

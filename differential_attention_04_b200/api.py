@@ -189,6 +189,48 @@ def diffattn_bwd_tc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch
     return dq, dk, dv, dlam, dw
 
 
+def rope_table(N: int, d: int, base: float = 10000.0, device=None) -> torch.Tensor:
+    """(cos, sin) of n * base^(-2j/d) for n < N, j < d/2: float32 [N, d/2, 2] on the device."""
+    t = torch.empty((N, d // 2, 2), dtype=torch.float32, device=device or torch.device("cuda"))
+    _check("diffattn_rope_table", lib().diffattn_rope_table(int(N), int(d), float(base), _ptr(t), _stream()))
+    return t
+
+
+def qkv_proj(x: torch.Tensor, w_qkv: torch.Tensor, B: int, N: int, H: int, d: int, rope: torch.Tensor | None = None,
+             out=None):
+    """[Q | K | V] = x w_qkv^T with RoPE (from rope_table) on Q and K: q, k [B, N, H, 2, d], v [B, N, H, 2d],
+    bfloat16.  x: bfloat16 [B*N, d_model]; w_qkv: bfloat16 [3*H*2d, d_model] (W_q; W_k; W_v)."""
+    _dev(x, w_qkv)
+    dm = x.shape[-1]
+    if x.dtype != torch.bfloat16 or w_qkv.dtype != torch.bfloat16 or x.numel() != B * N * dm:
+        raise ValueError("x must be bfloat16 [B*N, d_model]")
+    if tuple(w_qkv.shape) != (3 * H * 2 * d, dm):
+        raise ValueError("w_qkv must be bfloat16 [3*H*2d, d_model]")
+    if rope is not None and (rope.dtype != torch.float32 or rope.shape[0] < N or rope.shape[1] * 2 != d):
+        raise ValueError("rope must come from rope_table(>= N, d)")
+    if out is None:
+        bf = dict(dtype=torch.bfloat16, device=x.device)
+        out = (torch.empty((B, N, H, 2, d), **bf), torch.empty((B, N, H, 2, d), **bf), torch.empty((B, N, H, 2 * d), **bf))
+    q, k, v = out
+    _check("diffattn_qkv_proj", lib().diffattn_qkv_proj(
+        _ptr(x), _ptr(w_qkv), B, N, dm, H, d, _ptr(rope) if rope is not None else None, _ptr(q), _ptr(k), _ptr(v),
+        _stream()))
+    return q, k, v
+
+
+def out_proj(o: torch.Tensor, w_o: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = o w_o^T: o bfloat16 [M, K] (or [B, N, H, 2d]), w_o bfloat16 [n_out, K] -> y bfloat16 [M, n_out]."""
+    _dev(o, w_o)
+    K = w_o.shape[1]
+    if o.dtype != torch.bfloat16 or w_o.dtype != torch.bfloat16 or o.numel() % K:
+        raise ValueError("o and w_o must be bfloat16 with o's rows of width w_o.shape[1]")
+    M, n_out = o.numel() // K, w_o.shape[0]
+    if out is None:
+        out = torch.empty((M, n_out), dtype=torch.bfloat16, device=o.device)
+    _check("diffattn_out_proj", lib().diffattn_out_proj(_ptr(o), _ptr(w_o), M, K, n_out, _ptr(out), _stream()))
+    return out
+
+
 def diffattn_lambda_bwd(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor, lk2: torch.Tensor,
                         dlam: torch.Tensor):
     """Gradients (dlq1, dlk1, dlq2, dlk2) of the lambda re-parameterisation for a device dlambda."""

@@ -80,6 +80,20 @@ bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 
 bool fits_i32(long long x) { return x >= 0 && x < (1ll << 31); }
 
+// A projection GEMM through launch_proj_gemm, with the maps over A [M, K] and B [n_total, K].
+int proj_launch(const void* a, const void* b, int M, int K, int n_total, ProjParams& prm, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!encode_4d(&ta, a, K, 1, M, 1, 2, 128) || !encode_4d(&tb, b, K, 1, n_total, 1, 2, 256)) return DIFFATTN_ERR_CUDA;
+  DevCtl ctl;
+  if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  prm.M = M;
+  prm.N = n_total;
+  prm.K = K;
+  prm.status = ctl.status;
+  prm.limit_ns = g_wait_limit_ns.load();
+  return cuda_status(launch_proj_gemm(ta, tb, prm, stream));
+}
+
 }  // namespace
 }  // namespace diffattn
 
@@ -258,6 +272,57 @@ int diffattn_bwd_tc(const void* q, const void* k, const void* v, const void* dy,
   ctl.limit_ns = g_wait_limit_ns.load();
   return cuda_status(launch_bwd_sm100(m, dy, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv,
                                       dlambda, drms_w, workspace, ctl, stream));
+}
+
+int diffattn_rope_table(int seq_len, int d, double base, float* table, cudaStream_t stream) {
+  if (seq_len < 1 || d < 2 || d % 2 || !(base > 0.0) || !table) return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(seq_len) * d)) return DIFFATTN_ERR_INVALID_ARG;
+  return cuda_status(launch_rope_table(seq_len, d, base, table, stream));
+}
+
+
+int diffattn_qkv_proj(const void* x, const void* w_qkv, int B, int N, int d_model, int H, int d,
+                      const float* rope_table, void* q, void* k, void* v, cudaStream_t stream) {
+  if (B < 1 || N < 1 || d_model < 1 || H < 1 || d < 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (!x || !w_qkv || !q || !k || !v) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (rope_table && !aligned16(rope_table)))
+    return DIFFATTN_ERR_INVALID_ARG;
+  const long long hq = 2ll * H * d;
+  if (!fits_i32(static_cast<long long>(B) * N * d_model) || !fits_i32(3 * hq * d_model) ||
+      !fits_i32(static_cast<long long>(B) * N * 3 * hq))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (d_model % 64 || d % 32) return DIFFATTN_ERR_UNSUPPORTED;
+  ProjParams prm = {};
+  prm.seq_len = N;
+  prm.d = d;
+  prm.rope = reinterpret_cast<const float2*>(rope_table);
+  prm.rope_end = static_cast<int>(2 * hq);
+  prm.col_end[0] = static_cast<int>(hq);
+  prm.col_end[1] = static_cast<int>(2 * hq);
+  prm.col_end[2] = static_cast<int>(3 * hq);
+  prm.out[0] = static_cast<__nv_bfloat16*>(q);
+  prm.out[1] = static_cast<__nv_bfloat16*>(k);
+  prm.out[2] = static_cast<__nv_bfloat16*>(v);
+  return proj_launch(x, w_qkv, B * N, d_model, static_cast<int>(3 * hq), prm, stream);
+}
+
+int diffattn_out_proj(const void* o, const void* w_o, int M, int K, int n_out, void* y, cudaStream_t stream) {
+  if (M < 1 || K < 1 || n_out < 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (!o || !w_o || !y) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(y)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(M) * K) || !fits_i32(static_cast<long long>(n_out) * K) ||
+      !fits_i32(static_cast<long long>(M) * n_out))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (K % 64 || n_out % 32) return DIFFATTN_ERR_UNSUPPORTED;
+  ProjParams prm = {};
+  prm.seq_len = 1;
+  prm.d = 32;
+  prm.rope = nullptr;
+  prm.rope_end = 0;
+  prm.col_end[0] = prm.col_end[1] = prm.col_end[2] = n_out;
+  prm.out[0] = prm.out[1] = prm.out[2] = static_cast<__nv_bfloat16*>(y);
+  return proj_launch(o, w_o, M, K, n_out, prm, stream);
 }
 
 int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,

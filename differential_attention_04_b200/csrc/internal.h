@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -72,6 +73,26 @@ cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap&
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
                               const float* dlambda, float* dlq1, float* dlk1, float* dlq2, float* dlk2,
                               cudaStream_t stream);
+
+// Projection GEMM C[M, N] = A[M, K] B[N, K]^T (bf16, fp32 accumulation, bf16
+// out; K a multiple of 64, N and the column boundaries multiples of 32).
+// Columns [col_end[o-1], col_end[o]) go to out[o] (row stride = that width);
+// columns below rope_end get RoPE from `rope` (float2 cos/sin [seq_len][d/2])
+// at position (row mod seq_len) when rope is non-null.  ta maps A as
+// (K, 1, M, 1) with boxes of 64 x 128 rows, tb maps B as (K, 1, N, 1) with
+// boxes of 64 x 256 rows.
+struct ProjParams {
+  int M, N, K, seq_len, d, rope_end;
+  int col_end[3];
+  __nv_bfloat16* out[3];
+  const float2* rope;
+  int* status;
+  unsigned long long limit_ns;
+};
+cudaError_t launch_proj_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const ProjParams& prm,
+                             cudaStream_t stream);
+// cos/sin of n * base^(-2j/d) in double precision, rounded to float: [seq_len][d/2] float2.
+cudaError_t launch_rope_table(int seq_len, int d, double base, float* table, cudaStream_t stream);
 
 // Split-KV decode (bf16, d = 128).
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);

@@ -15,6 +15,11 @@ no dataset or trained weight is used):
   * Needle (long-context case): for every head h of every batch b, at a seeded
     position p < N-1, K1[b, p, h] = 4 * Q1[b, N-1, h] / |Q1[b, N-1, h]|
     (computed in float32 from the stored query, then rounded); K2 stays noise.
+  * Projections (the steps either side of the path): token activations X
+    i.i.d. N(0, 1) [B*N, d_model]; weights i.i.d. N(0, 1/d_model) (so the
+    projected entries have unit variance), drawn like Q, K, V and rounded to
+    bf16: W_qkv [3 * H * 2d, d_model], W_o [d_model, H * 2d].  The 3B-like
+    model: d_model = 3072, H = 12, d = 128.
   * Decode: per-sequence KV length L_s ~ U{lmin .. lmax} from
     ``numpy.random.default_rng(seed).integers(lmin, lmax + 1, S)``; sequences
     packed back to back; the cache includes the current token.
@@ -150,3 +155,34 @@ def make_decode_case(name: str, seed=0, device="cpu", **override) -> DecodeInput
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact float64 copy (on the host) of a float32/bf16 tensor."""
     return t.detach().to("cpu", torch.float64).numpy()
+
+
+PROJ_CASES = {
+    "proj_3b": dict(B=4, N=4096, d_model=3072, H=12, d=128),
+}
+
+
+@dataclass
+class ProjInputs:
+    x: torch.Tensor      # [B*N, d_model]
+    w_qkv: torch.Tensor  # [3 * H * 2d, d_model]
+    w_o: torch.Tensor    # [d_model, H * 2d]
+    B: int
+    N: int
+    H: int
+    d: int
+
+
+def make_proj(B, N, d_model, H, d, seed=0, device="cpu") -> ProjInputs:
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = _randn((B * N, d_model), gen, device, torch.bfloat16)
+    w_qkv = _randn((3 * H * 2 * d, d_model), gen, device, torch.float32)
+    w_qkv = (w_qkv / float(np.sqrt(d_model))).to(torch.bfloat16)
+    w_o = _randn((d_model, H * 2 * d), gen, device, torch.float32)
+    w_o = (w_o / float(np.sqrt(H * 2 * d))).to(torch.bfloat16)
+    return ProjInputs(x, w_qkv, w_o, B, N, H, d)
+
+
+def make_proj_case(name: str, seed=0, device="cpu") -> ProjInputs:
+    return make_proj(seed=seed, device=device, **PROJ_CASES[name])

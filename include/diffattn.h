@@ -197,6 +197,44 @@ int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2,
                         cudaStream_t stream);
 
 /*
+ * The steps either side of the path (page "Differential attention", "How it's
+ * wired (and why it's nearly free)": each head's query and key projections
+ * split into halves Q1, K1 and Q2, K2; the layer sits in a standard
+ * transformer block).  Rotary position embedding as in RoFormer (cited on
+ * page "Differential Transformer", "Builds on"): consecutive channel pairs
+ * (2j, 2j+1) of every d-wide Q1, Q2, K1, K2 rotated by the angle
+ * n * base^(-2j/d) at the token's position n within its sequence.
+ *
+ * diffattn_rope_table -- table[n][j] = (cos, sin) of n * base^(-2j/d),
+ *   computed in double precision and rounded to float32.
+ *   table : device float32 [seq_len][d/2][2], written.  d even, seq_len >= 1.
+ * diffattn_qkv_proj -- [Q | K | V] = X W_qkv^T on the tensor cores (fp32
+ *   accumulation), RoPE applied to Q and K in the same kernel's epilogue,
+ *   rounded to bf16 and written in the layouts diffattn_fwd reads:
+ *   x      : device bf16 [B * N, d_model] (rows: batch-major tokens)
+ *   w_qkv  : device bf16 [H*2*d + H*2*d + H*2d, d_model], a linear layer's
+ *            weight (one row per output feature): W_q, then W_k, then W_v;
+ *            W_q's rows ordered (head, map, channel), W_v's (head, channel)
+ *   rope_table : from diffattn_rope_table for at least N positions, or NULL
+ *            for no rotation
+ *   q, k   : device bf16 [B, N, H, 2, d], written;  v : [B, N, H, 2d], written
+ *   d_model a multiple of 64; d a multiple of 32.
+ * diffattn_out_proj -- y[M, n_out] = o[M, K] w_o[n_out, K]^T (bf16 in and out,
+ *   fp32 accumulation): the output projection of the heads' concatenated
+ *   outputs (o = diffattn_fwd's output viewed as [B * N, H * 2d]).
+ *   K a multiple of 64, n_out a multiple of 32.
+ * All pointers 16-byte aligned; stream-ordered; no allocation.
+ * Errors: DIFFATTN_ERR_INVALID_ARG (null or unaligned pointers, sizes),
+ * DIFFATTN_ERR_UNSUPPORTED (sizes outside the multiples above),
+ * DIFFATTN_ERR_CUDA; DIFFATTN_ERR_TIMEOUT through diffattn_device_status.
+ */
+int diffattn_rope_table(int seq_len, int d, double base, float* table, cudaStream_t stream);
+int diffattn_qkv_proj(const void* x, const void* w_qkv, int B, int N, int d_model, int H, int d,
+                      const float* rope_table, void* q, void* k, void* v, cudaStream_t stream);
+int diffattn_out_proj(const void* o, const void* w_o, int M, int K, int n_out, void* y,
+                      cudaStream_t stream);
+
+/*
  * Low-bit queries and keys (peer review "Differential Transformer",
  * Strengths, the activation-outlier bullet, and Questions, the quantisation
  * bullet: absmax quantisation per logit map and per head).

@@ -113,6 +113,23 @@ def test_validation_without_gpu(L):
     assert L.diffattn_bwd_tc_workspace_size(2, 300, 3, 128) == up(4 * 600 * 3 * 2 * 256) + up(2 * 600 * 3 * 256) + \
         up(16 * 2 * 3 * 384)
     assert L.diffattn_bwd_tc_workspace_size(1, 0, 2, 64) == 0
+    # projections: sizes, multiples, pointers
+    assert L.diffattn_rope_table(0, 64, 1e4, fake, nul) == api.ERR_INVALID_ARG
+    assert L.diffattn_rope_table(16, 7, 1e4, fake, nul) == api.ERR_INVALID_ARG
+    assert L.diffattn_rope_table(16, 64, -1.0, fake, nul) == api.ERR_INVALID_ARG
+    assert L.diffattn_rope_table(16, 64, 1e4, nul, nul) == api.ERR_INVALID_ARG
+    qp = lambda x, dm, d, rope=None: L.diffattn_qkv_proj(x, x, 2, 16, dm, 2, d, rope, x, x, x, nul)
+    assert qp(fake, 96, 64) == api.ERR_UNSUPPORTED     # d_model not a multiple of 64
+    assert qp(fake, 128, 48) == api.ERR_UNSUPPORTED    # d not a multiple of 32
+    assert qp(nul, 128, 64) == api.ERR_INVALID_ARG
+    assert qp(ctypes.c_void_p(4104), 128, 64) == api.ERR_INVALID_ARG
+    assert qp(fake, 128, 64, rope=ctypes.c_void_p(4100)) == api.ERR_INVALID_ARG
+    assert L.diffattn_qkv_proj(fake, fake, 0, 16, 128, 2, 64, nul, fake, fake, fake, nul) == api.ERR_INVALID_ARG
+    op = lambda x, M, K, n: L.diffattn_out_proj(x, x, M, K, n, x, nul)
+    assert op(fake, 16, 96, 64) == api.ERR_UNSUPPORTED
+    assert op(fake, 16, 128, 48) == api.ERR_UNSUPPORTED
+    assert op(fake, 0, 128, 64) == api.ERR_INVALID_ARG
+    assert op(nul, 16, 128, 64) == api.ERR_INVALID_ARG
     # decode
     dec = lambda q, d, ws, wsb, S=4: L.diffattn_decode(q, q, q, q, 100, q, S, 2, d, q, 0.5, q, 1e-5, ws, wsb, nul)
     assert dec(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG

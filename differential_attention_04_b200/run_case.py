@@ -4,6 +4,8 @@
   python -m differential_attention_04_b200.run_case prefill --qk8 1 ...   (e4m3 queries/keys: quantise + forward;
                                                                           2: forward only; 3: quantise only)
   python -m differential_attention_04_b200.run_case bwd --tc 1 ...   (tensor-core backward; 0: CUDA cores)
+  python -m differential_attention_04_b200.run_case proj --B 1 --N 4096 --H 12 --d 128 --dmodel 3072 --iters 3
+                                                                          (QKV projection + RoPE, then output projection)
   python -m differential_attention_04_b200.run_case decode --S 64 --H 12 --lmin 1024 --lmax 4096 --iters 3
 
 Inputs come from the seeded generators in ``workloads``; the output is not
@@ -22,7 +24,7 @@ from .build import build
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kind", choices=["prefill", "decode", "bwd"])
+    ap.add_argument("kind", choices=["prefill", "decode", "bwd", "proj"])
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--H", type=int, default=12)
@@ -31,6 +33,7 @@ def main(argv=None):
     ap.add_argument("--dtype", default="bf16")
     ap.add_argument("--qk8", type=int, default=0)
     ap.add_argument("--tc", type=int, default=1)
+    ap.add_argument("--dmodel", type=int, default=3072)
     ap.add_argument("--S", type=int, default=64)
     ap.add_argument("--lmin", type=int, default=1024)
     ap.add_argument("--lmax", type=int, default=4096)
@@ -70,6 +73,15 @@ def main(argv=None):
             ws = torch.empty(api.bwd_workspace_size(a.B, a.N, a.H, a.d), dtype=torch.uint8, device=dev)
             run = lambda: api.diffattn_bwd(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps,
                                            inp.causal, workspace=ws)
+    elif a.kind == "proj":
+        inp = wl.make_proj(a.B, a.N, a.dmodel, a.H, a.d, seed=a.seed, device=dev)
+        table = api.rope_table(a.N, a.d)
+        qkv = api.qkv_proj(inp.x, inp.w_qkv, a.B, a.N, a.H, a.d, table)
+        y = torch.empty((a.B * a.N, a.dmodel), dtype=torch.bfloat16, device=dev)
+
+        def run():
+            api.qkv_proj(inp.x, inp.w_qkv, a.B, a.N, a.H, a.d, table, out=qkv)
+            api.out_proj(qkv[2], inp.w_o, out=y)
     else:
         inp = wl.make_decode(a.S, a.H, a.d, a.lmin, a.lmax, seed=a.seed, device=dev)
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)

@@ -26,7 +26,7 @@ What it computes, and where the pages define it
 * The row max is subtracted before exponentiating (the softmax in the worked
   example on page "Differential attention", "The noise-canceling idea").
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   d in sqrt(d) is the per-map query/key width; eps sits inside the square
   root; w is one fp32 vector of length 2d shared by all heads; the scale uses
   lambda_init (not the learned lambda) and is applied after w; causal means key

@@ -222,6 +222,13 @@ __global__ void __launch_bounds__(kGradThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kColTile, false, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, KIND == kGradV ? C::DV : D, false, true);
       const uint32_t sRa = smem_u32(sR), sCa = smem_u32(sC);
+      // Descriptors are built once and advanced by adding (offset >> 4) to
+      // their address field: the issue queue holds about one instruction, so
+      // address arithmetic between two products would delay the second.
+      const uint64_t a_desc = smem_desc_sw128(sRa, 16, 1024);
+      const uint64_t c_desc = smem_desc_sw128(sCa, 16, 1024);             // K-major column tiles
+      const uint64_t c_desc_mn = smem_desc_sw128(sCa, C::CBOX, 1024);     // the same tiles read MN-major
+      auto adv = [](uint64_t desc, uint32_t bytes) { return desc + static_cast<uint64_t>(bytes >> 4); };
       bool ok = mbar_wait(&bars->r_full, 0, wc);
       // S of tile i is issued before the gradient product of tile i - 1, so
       // that the tensor core works on tile i while the softmax warps turn
@@ -233,26 +240,22 @@ __global__ void __launch_bounds__(kGradThreads, 1)
           if (!(ok = mbar_wait(&bars->c_full[st], (i / C::STAGES) & 1, wc))) break;
           tc_fence_after();
           const uint32_t tb = tmem + C::TM_BUF + 128u * bb;
-          const uint32_t cb = sCa + st * C::C_BYTES;
+          const uint64_t cd = adv(c_desc, st * C::C_BYTES);
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const int blk = kk >> 2;
-              const uint32_t koff = (kk & 3) * 32;
-              const uint64_t ad = smem_desc_sw128(sRa + (m * C::QKB + blk) * C::RBOX + koff, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(cb + (m * C::QKB + blk) * C::CBOX + koff, 16, 1024);
-              umma_ss(tb + (m ? C::B_S2 : C::B_S1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+              const uint32_t blk = kk >> 2, koff = (kk & 3) * 32;
+              umma_ss(tb + (m ? C::B_S2 : C::B_S1), adv(a_desc, (m * C::QKB + blk) * C::RBOX + koff),
+                      adv(cd, (m * C::QKB + blk) * C::CBOX + koff), idesc_s, kk > 0 ? 1u : 0u);
             }
           }
           if constexpr (C::HAS_DP) {
 #pragma unroll
             for (int kk = 0; kk < C::DV / 16; ++kk) {
-              const int blk = kk >> 2;
-              const uint32_t koff = (kk & 3) * 32;
-              const uint64_t ad = smem_desc_sw128(sRa + C::R_QK + blk * C::RBOX + koff, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(cb + C::C_QK + blk * C::CBOX + koff, 16, 1024);
-              umma_ss(tb + C::B_DP, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+              const uint32_t blk = kk >> 2, koff = (kk & 3) * 32;
+              umma_ss(tb + C::B_DP, adv(a_desc, C::R_QK + blk * C::RBOX + koff), adv(cd, C::C_QK + blk * C::CBOX + koff),
+                      idesc_s, kk > 0 ? 1u : 0u);
             }
           }
           umma_commit(&bars->s_full[bb]);
@@ -262,23 +265,20 @@ __global__ void __launch_bounds__(kGradThreads, 1)
           if (!(ok = mbar_wait(&bars->a_full[bj], (j >> 1) & 1, wc))) break;
           tc_fence_after();
           const uint32_t tb = tmem + C::TM_BUF + 128u * bj;
-          const uint32_t cb = sCa + stj * C::C_BYTES;
+          const uint64_t cd = adv(c_desc_mn, stj * C::C_BYTES);
           // B operands: the stage's rows [32][width] read MN-major (K = the 32 columns)
           if constexpr (KIND == kGradV) {
 #pragma unroll
-            for (int kk = 0; kk < kColTile / 16; ++kk) {
-              const uint64_t bd = smem_desc_sw128(cb + C::C_QK + kk * 2048, C::CBOX, 1024);
-              umma_ts(tmem + C::TM_ACC, tb + C::B_A1 + 8 * kk, bd, idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < kColTile / 16; ++kk)
+              umma_ts(tmem + C::TM_ACC, tb + C::B_A1 + 8 * kk, adv(cd, C::C_QK + kk * 2048), idesc_g,
+                      (j > 0 || kk > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
 #pragma unroll
-              for (int kk = 0; kk < kColTile / 16; ++kk) {
-                const uint64_t bd = smem_desc_sw128(cb + m * C::QKB * C::CBOX + kk * 2048, C::CBOX, 1024);
-                umma_ts(tmem + C::TM_ACC + m * D, tb + (m ? C::B_A2 : C::B_A1) + 8 * kk, bd, idesc_g,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-              }
+              for (int kk = 0; kk < kColTile / 16; ++kk)
+                umma_ts(tmem + C::TM_ACC + m * D, tb + (m ? C::B_A2 : C::B_A1) + 8 * kk,
+                        adv(cd, m * C::QKB * C::CBOX + kk * 2048), idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(&bars->c_empty[stj]);  // S_j and the gradient product of tile j have read the stage

@@ -291,8 +291,39 @@ def bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, K):
     sustained = loop_ms >= 1000.0
     peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     achieved = alg / (ms * 1e-3) / 1e12
+
+    # the training pair: a forward that saves the statistics, and the backward that uses them
+    y = torch.empty_like(inp.v)
+
+    def fwd_train():
+        api.diffattn_fwd_train(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
+                               workspace=ws, out=y)
+
+    def bwd_saved():
+        api.diffattn_bwd_tc_saved(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal,
+                                  api.MODE_DIFF, ws, out=outs)
+
+    for _ in range(3):
+        fwd_train()
+        bwd_saved()
+    torch.cuda.synchronize()
+    barrier()
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for e0, e1, e2 in ev2:
+        e0.record()
+        fwd_train()
+        e1.record()
+        bwd_saved()
+        e2.record()
+    torch.cuda.synchronize()
+    ft_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b, _ in ev2))
+    bs_ms = reduce_max(statistics.mean(b.elapsed_time(c) for _, b, c in ev2))
     return {"metric": "DiffAttn backward TFLOP/s (dq, dk, dv, dlambda, dw)", "value": achieved, "unit": "TFLOP/s",
             "steps": K, "ms_per_step": ms, "flops_per_step_algorithmic": alg, "flops_per_step_executed": executed,
+            "training_pair": {"fwd_train_ms": ft_ms, "bwd_saved_ms": bs_ms,
+                              "bwd_saved_tflops_algorithmic": alg / (bs_ms * 1e-3) / 1e12,
+                              "note": "diffattn_fwd_train (output + each map's A_i V and log-sum-exp) then "
+                                      "diffattn_bwd_tc_saved (no statistics pass)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None,
                          "executed_tflops": executed / (ms * 1e-3) / 1e12,
@@ -300,7 +331,7 @@ def bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, K):
                          "peak_source": f"{peak_src} bf16 dense, " + (
                              f"sustained (timed loop {loop_ms / 1e3:.2f} s)" if sustained
                              else f"burst (timed loop {loop_ms / 1e3:.2f} s)")},
-            "gpu_launches": 5 * K}
+            "gpu_launches": 10 * K}
 
 
 def bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, K):

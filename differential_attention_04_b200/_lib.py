@@ -30,6 +30,10 @@ SIGNATURES = {
     "diffattn_bwd_tc_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_bwd_tc": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
                                  _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "diffattn_fwd_train": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float, _vp,
+                                    _c_float, _c_int, _vp, _c_size, _vp]),
+    "diffattn_bwd_tc_saved": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
+                                       _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "diffattn_rope_table": (_c_int, [_c_int, _c_int, ctypes.c_double, _vp, _vp]),
     "diffattn_qkv_proj": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "diffattn_out_proj": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp]),

@@ -189,6 +189,49 @@ def diffattn_bwd_tc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch
     return dq, dk, dv, dlam, dw
 
 
+def diffattn_fwd_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor, lambda_init: float,
+                       rms_w: torch.Tensor, eps: float = 1e-5, causal: bool = True, mode: int = MODE_DIFF,
+                       workspace: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """Training forward: (o, workspace).  o as diffattn_fwd; the workspace (bwd_tc_workspace_size bytes) holds
+    what diffattn_bwd_tc_saved needs for the same q, k, v, lambda and mask."""
+    _dev(q, k, v, lam, rms_w)
+    B, N, H, two, d = q.shape
+    if two != 2 or k.shape != q.shape or tuple(v.shape) != (B, N, H, 2 * d):
+        raise ValueError("shapes must be q, k: [B, N, H, 2, d] and v: [B, N, H, 2d]")
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v)):
+        raise ValueError("q, k, v must be bfloat16")
+    if out is None:
+        out = torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(bwd_tc_workspace_size(B, N, H, d), dtype=torch.uint8, device=q.device)
+    _check("diffattn_fwd_train", lib().diffattn_fwd_train(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+        _ptr(rms_w), float(eps), int(mode), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()))
+    return out, workspace
+
+
+def diffattn_bwd_tc_saved(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch.Tensor, lam: torch.Tensor,
+                          lambda_init: float, rms_w: torch.Tensor, eps: float, causal: bool, mode: int,
+                          workspace: torch.Tensor, out=None):
+    """diffattn_bwd_tc using the statistics diffattn_fwd_train left in `workspace`."""
+    _dev(q, k, v, dy, lam, rms_w, workspace)
+    B, N, H, two, d = q.shape
+    if two != 2 or k.shape != q.shape or tuple(v.shape) != (B, N, H, 2 * d) or dy.shape != v.shape:
+        raise ValueError("shapes must be q, k: [B, N, H, 2, d] and v, dy: [B, N, H, 2d]")
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, dy)):
+        raise ValueError("q, k, v, dy must be bfloat16")
+    if out is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        out = (torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32),
+               torch.empty(1, **f32), torch.empty(2 * d, **f32))
+    dq, dk, dv, dlam, dw = out
+    _check("diffattn_bwd_tc_saved", lib().diffattn_bwd_tc_saved(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dy), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+        _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream()))
+    return dq, dk, dv, dlam, dw
+
+
 def rope_table(N: int, d: int, base: float = 10000.0, device=None) -> torch.Tensor:
     """(cos, sin) of n * base^(-2j/d) for n < N, j < d/2: float32 [N, d/2, 2] on the device."""
     t = torch.empty((N, d // 2, 2), dtype=torch.float32, device=device or torch.device("cuda"))

@@ -94,6 +94,39 @@ int proj_launch(const void* a, const void* b, int M, int K, int n_total, ProjPar
   return cuda_status(launch_proj_gemm(ta, tb, prm, stream));
 }
 
+// diffattn_bwd_tc and diffattn_bwd_tc_saved: the same checks and maps; `saved`
+// skips the statistics pass (the workspace already holds them).
+int bwd_tc_impl(const void* q, const void* k, const void* v, const void* dy, int B, int N, int H, int d, int causal,
+                const float* lambda, float lambda_init, const float* rms_w, float eps, int mode, float* dq, float* dk,
+                float* dv, float* dlambda, float* drms_w, void* workspace, size_t ws_bytes, bool saved,
+                cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !dy || !lambda || !rms_w || !dq || !dk || !dv || !dlambda || !drms_w)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * ((N + 127) / 128) > 0x7fffffffll) return DIFFATTN_ERR_UNSUPPORTED;
+  const BwdTcLayout L = bwd_tc_layout(B, N, H, d);
+  if (!workspace || ws_bytes < L.bytes || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
+  const void* g = static_cast<const char*>(workspace) + L.off_g;
+  BwdTcMaps m;
+  if (!encode_4d(&m.q128, q, d, 2ull * H, N, B) || !encode_4d(&m.q32, q, d, 2ull * H, N, B, 2, 32) ||
+      !encode_4d(&m.k128, k, d, 2ull * H, N, B) || !encode_4d(&m.k32, k, d, 2ull * H, N, B, 2, 32) ||
+      !encode_4d(&m.v128, v, 2ull * d, H, N, B) || !encode_4d(&m.v32, v, 2ull * d, H, N, B, 2, 32) ||
+      !encode_4d(&m.g128, g, 2ull * d, H, N, B) || !encode_4d(&m.g32, g, 2ull * d, H, N, B, 2, 32))
+    return DIFFATTN_ERR_CUDA;
+  DevCtl ctl;
+  if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  ctl.limit_ns = g_wait_limit_ns.load();
+  return cuda_status(launch_bwd_sm100(m, dy, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv,
+                                      dlambda, drms_w, workspace, saved, ctl, stream));
+}
 }  // namespace
 }  // namespace diffattn
 
@@ -242,36 +275,47 @@ size_t diffattn_bwd_tc_workspace_size(int B, int N, int H, int d) {
   return bwd_tc_layout(B, N, H, d).bytes;
 }
 
+
 int diffattn_bwd_tc(const void* q, const void* k, const void* v, const void* dy, int B, int N, int H, int d,
                     int causal, const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                     float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
                     size_t ws_bytes, cudaStream_t stream) {
+  return bwd_tc_impl(q, k, v, dy, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv, dlambda,
+                     drms_w, workspace, ws_bytes, false, stream);
+}
+
+int diffattn_bwd_tc_saved(const void* q, const void* k, const void* v, const void* dy, int B, int N, int H, int d,
+                          int causal, const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                          float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
+                          size_t ws_bytes, cudaStream_t stream) {
+  return bwd_tc_impl(q, k, v, dy, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv, dlambda,
+                     drms_w, workspace, ws_bytes, true, stream);
+}
+
+int diffattn_fwd_train(const void* q, const void* k, const void* v, void* o, int B, int N, int H, int d, int causal,
+                       const float* lambda, float lambda_init, const float* rms_w, float eps, int mode, void* workspace,
+                       size_t ws_bytes, cudaStream_t stream) {
   if (B < 1 || H < 1 || N < 1 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
   if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
     return DIFFATTN_ERR_INVALID_ARG;
   if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
-  if (!q || !k || !v || !dy || !lambda || !rms_w || !dq || !dk || !dv || !dlambda || !drms_w)
-    return DIFFATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
-      !aligned16(dv))
-    return DIFFATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lambda || !rms_w) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DIFFATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H * ((N + 127) / 128) > 0x7fffffffll) return DIFFATTN_ERR_UNSUPPORTED;
   const BwdTcLayout L = bwd_tc_layout(B, N, H, d);
   if (!workspace || ws_bytes < L.bytes || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
-  const void* g = static_cast<const char*>(workspace) + L.off_g;
-  BwdTcMaps m;
-  if (!encode_4d(&m.q128, q, d, 2ull * H, N, B) || !encode_4d(&m.q32, q, d, 2ull * H, N, B, 2, 32) ||
-      !encode_4d(&m.k128, k, d, 2ull * H, N, B) || !encode_4d(&m.k32, k, d, 2ull * H, N, B, 2, 32) ||
-      !encode_4d(&m.v128, v, 2ull * d, H, N, B) || !encode_4d(&m.v32, v, 2ull * d, H, N, B, 2, 32) ||
-      !encode_4d(&m.g128, g, 2ull * d, H, N, B) || !encode_4d(&m.g32, g, 2ull * d, H, N, B, 2, 32))
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
+      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
-  return cuda_status(launch_bwd_sm100(m, dy, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv,
-                                      dlambda, drms_w, workspace, ctl, stream));
+  char* ws = static_cast<char*>(workspace);
+  return cuda_status(launch_prefill_sm100_stats(tq, tk, tv, &to, o, B, N, H, d, causal, lambda, lambda_init, rms_w,
+                                                eps, mode, reinterpret_cast<float*>(ws + L.off_omaps),
+                                                reinterpret_cast<float*>(ws + L.off_stats), L.n_pad, ctl, stream));
 }
 
 int diffattn_rope_table(int seq_len, int d, double base, float* table, cudaStream_t stream) {

@@ -516,7 +516,7 @@ template <int D>
 cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N, int H, int causal,
                                const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                                float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
-                               DevCtl ctl, cudaStream_t stream) {
+                               bool stats_ready, DevCtl ctl, cudaStream_t stream) {
   const BwdTcLayout L = bwd_tc_layout(B, N, H, D);
   char* ws = static_cast<char*>(workspace);
   float* o_maps = reinterpret_cast<float*>(ws + L.off_omaps);
@@ -525,9 +525,11 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   cudaError_t e = cudaMemsetAsync(drms_w, 0, sizeof(float) * 2 * D, stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(dlambda, 0, sizeof(float), stream);
   if (e != cudaSuccess) return e;
-  e = launch_prefill_sm100_stats(m.q128, m.k128, m.v128, B, N, H, D, causal, lambda, o_maps,
-                                 reinterpret_cast<float*>(stats), L.n_pad, ctl, stream);
-  if (e != cudaSuccess) return e;
+  if (!stats_ready) {
+    e = launch_prefill_sm100_stats(m.q128, m.k128, m.v128, nullptr, nullptr, B, N, H, D, causal, lambda, lambda_init,
+                                   rms_w, eps, mode, o_maps, reinterpret_cast<float*>(stats), L.n_pad, ctl, stream);
+    if (e != cudaSuccess) return e;
+  }
   const long long rows = static_cast<long long>(B) * N * H;
   const long long want = (rows + 7) / 8;
   const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
@@ -577,13 +579,13 @@ BwdTcLayout bwd_tc_layout(int B, int N, int H, int d) {
 cudaError_t launch_bwd_sm100(const BwdTcMaps& m, const void* dy, int B, int N, int H, int d, int causal,
                              const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                              float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
-                             DevCtl ctl, cudaStream_t stream) {
+                             bool stats_ready, DevCtl ctl, cudaStream_t stream) {
   if (d == 128)
     return launch_bwd_sm100_d<128>(m, dy, B, N, H, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv,
-                                   dlambda, drms_w, workspace, ctl, stream);
+                                   dlambda, drms_w, workspace, stats_ready, ctl, stream);
   if (d == 64)
     return launch_bwd_sm100_d<64>(m, dy, B, N, H, causal, lambda, lambda_init, rms_w, eps, mode, dq, dk, dv,
-                                  dlambda, drms_w, workspace, ctl, stream);
+                                  dlambda, drms_w, workspace, stats_ready, ctl, stream);
   return cudaErrorInvalidValue;
 }
 

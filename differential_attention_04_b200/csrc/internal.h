@@ -61,15 +61,19 @@ struct BwdTcLayout {
   int n_pad;
 };
 BwdTcLayout bwd_tc_layout(int B, int N, int H, int d);
+// stats_ready: the workspace already holds the statistics (from the training
+// forward with the same q, k, v, lambda and mask): the statistics pass is skipped.
 cudaError_t launch_bwd_sm100(const BwdTcMaps& m, const void* dy, int B, int N, int H, int d, int causal,
                              const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                              float* dq, float* dk, float* dv, float* dlambda, float* drms_w, void* workspace,
-                             DevCtl ctl, cudaStream_t stream);
+                             bool stats_ready, DevCtl ctl, cudaStream_t stream);
 // The tcgen05 prefill in its statistics mode: per map, O_i / l_i into
-// o_maps and the log2-sum-exp into component i of the float4 rows of lse.
-cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, int B,
-                                       int N, int H, int d, int causal, const float* lambda, float* o_maps,
-                                       float* lse, int n_pad, DevCtl ctl, cudaStream_t stream);
+// o_maps and the log2-sum-exp into component i of the float4 rows of lse;
+// with `to` (the output map over o) non-null, the normalised output too.
+cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                       const CUtensorMap* to, void* o, int B, int N, int H, int d, int causal,
+                                       const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                                       float* o_maps, float* lse, int n_pad, DevCtl ctl, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
                               const float* dlambda, float* dlq1, float* dlk1, float* dlq2, float* dlk2,
                               cudaStream_t stream);

@@ -151,9 +151,12 @@ __device__ __forceinline__ void tmem_ld_wait4(uint32_t (&a)[32], uint32_t (&b)[3
   tmem_ld_wait(d);
 }
 
-// STATS: instead of the normalised output, each CTA writes its own map's
-// O_i / l_i (float32) and log-sum-exp, for the backward pass.
-template <int D, bool QK8, bool STATS>
+// OUT selects what the epilogue writes: kOutNorm the normalised output;
+// kOutStats instead of it, each CTA's own map's O_i / l_i (float32) and
+// log-sum-exp (what the backward pass needs); kOutBoth both (a training
+// forward that saves the backward's statistics).
+enum : int { kOutNorm = 0, kOutStats = 1, kOutBoth = 2 };
+template <int D, bool QK8, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                          const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -501,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O is complete once the item's last PV (and with it every earlier MMA) has.
       if (sm_ok) sm_ok = mbar_wait(&bars->p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, wc);
       tc_fence_after();
-      if constexpr (STATS) {
+      if constexpr (OUT != kOutNorm) {
         // This map's O_i / l_i for the row, and lse_i = m + log2(l) in the
         // scaled log2 units of P = exp2(s * sc - m): P / l = exp2(s * sc - lse_i).
         const bool live = qrow < N;
@@ -521,11 +524,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (live) p.lse[((static_cast<size_t>(it.b) * p.H + it.h) * p.n_pad + qrow) * 4 + rank] = m_run + log2f(l_run);
-        tc_fence_before();
-        named_bar_sync(1, 128);  // every row's tensor-memory reads are done
-        if (tid == 128) mbar_arrive(&bars->epi_free);  // the next item's first PV may overwrite O
-        __syncwarp();
-        continue;
+        if constexpr (OUT == kOutStats) {
+          tc_fence_before();
+          named_bar_sync(1, 128);  // every row's tensor-memory reads are done
+          if (tid == 128) mbar_arrive(&bars->epi_free);  // the next item's first PV may overwrite O
+          __syncwarp();
+          continue;
+        }
+        // kOutBoth: O is still in tensor memory (the next item's first PV waits for epi_free)
       }
       // Both V stages are free of this item's PV products: announce that this
       // CTA's receive buffer is ready, with the exchange barrier armed first.
@@ -625,11 +631,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool QK8, bool STATS = false>
+template <int D, bool QK8, int OUT = kOutNorm>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const PrefillParams& prm, cudaStream_t stream) {
   using C = Cfg<D, QK8>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8, STATS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -651,12 +657,12 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if (mc == 0) {
     cfg.gridDim = dim3(2 * 128, 1, 1);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QK8, STATS>, &cfg) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QK8, OUT>, &cfg) != cudaSuccess || n < 1) n = 1;
     mc = n;
   }
   const int clusters = prm.n_items < mc ? prm.n_items : mc;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8, STATS>, tq, tk, tv, to, prm);
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8, OUT>, tq, tk, tv, to, prm);
 }
 
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -693,10 +699,12 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, int B,
-                                       int N, int H, int d, int causal, const float* lambda, float* o_maps,
-                                       float* lse, int n_pad, DevCtl ctl, cudaStream_t stream) {
+cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                       const CUtensorMap* to, void* o, int B, int N, int H, int d, int causal,
+                                       const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                                       float* o_maps, float* lse, int n_pad, DevCtl ctl, cudaStream_t stream) {
   PrefillParams prm = {};
+  prm.o = static_cast<__nv_bfloat16*>(o);
   prm.N = N;
   prm.H = H;
   prm.B = B;
@@ -709,17 +717,23 @@ cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap&
     prm.head_group = static_cast<int>(grp < 1 ? 1 : (grp > B * H ? B * H : grp));
   }
   prm.lambda = lambda;
-  prm.mode = 0;
-  prm.lambda_init = 0.f;
-  prm.eps = 1.f;
+  prm.mode = mode;
+  prm.lambda_init = lambda_init;
+  prm.rms_w = rms_w;
+  prm.eps = eps;
   prm.status = ctl.status;
   prm.limit_ns = ctl.limit_ns;
   prm.o_maps = o_maps;
   prm.lse = lse;
   prm.n_pad = n_pad;
-  // the output map is never used in this mode: tv stands in for it
-  if (d == 128) return launch_d<128, false, true>(tq, tk, tv, tv, prm, stream);
-  if (d == 64) return launch_d<64, false, true>(tq, tk, tv, tv, prm, stream);
+  if (to) {  // the normalised output as well
+    if (d == 128) return launch_d<128, false, kOutBoth>(tq, tk, tv, *to, prm, stream);
+    if (d == 64) return launch_d<64, false, kOutBoth>(tq, tk, tv, *to, prm, stream);
+    return cudaErrorInvalidValue;
+  }
+  // statistics only: the output map is never used, tv stands in for it
+  if (d == 128) return launch_d<128, false, kOutStats>(tq, tk, tv, tv, prm, stream);
+  if (d == 64) return launch_d<64, false, kOutStats>(tq, tk, tv, tv, prm, stream);
   return cudaErrorInvalidValue;
 }
 

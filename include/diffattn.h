@@ -178,6 +178,31 @@ int diffattn_bwd(const void* q, const void* k, const void* v, const void* dy,
  * diffattn_device_status if a kernel wait ran out.
  */
 size_t diffattn_bwd_tc_workspace_size(int B, int N, int H, int d);
+
+/*
+ * Training pair: a forward that also saves what the tensor-core backward
+ * needs, and the backward that uses it instead of recomputing it.
+ *
+ * diffattn_fwd_train -- diffattn_fwd_mode's output o (bf16, d = 64 or 128),
+ *   and into `workspace` (>= diffattn_bwd_tc_workspace_size bytes) each map's
+ *   A_i V (float32) and the log-sum-exp of every query row.  Other arguments
+ *   and errors as in diffattn_fwd_mode; DIFFATTN_ERR_WORKSPACE as below.
+ * diffattn_bwd_tc_saved -- diffattn_bwd_tc without its statistics pass: the
+ *   workspace must hold what diffattn_fwd_train wrote for the same q, k, v,
+ *   lambda and mask (the mode may differ: the statistics do not depend on it).
+ *   Arguments, outputs and errors as in diffattn_bwd_tc.
+ */
+int diffattn_fwd_train(const void* q, const void* k, const void* v, void* o,
+                       int B, int N, int H, int d, int causal,
+                       const float* lambda, float lambda_init, const float* rms_w,
+                       float eps, int mode, void* workspace, size_t ws_bytes,
+                       cudaStream_t stream);
+int diffattn_bwd_tc_saved(const void* q, const void* k, const void* v, const void* dy,
+                          int B, int N, int H, int d, int causal,
+                          const float* lambda, float lambda_init, const float* rms_w,
+                          float eps, int mode, float* dq, float* dk, float* dv,
+                          float* dlambda, float* drms_w, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream);
 int diffattn_bwd_tc(const void* q, const void* k, const void* v, const void* dy,
                     int B, int N, int H, int d, int causal,
                     const float* lambda, float lambda_init, const float* rms_w,

@@ -113,6 +113,19 @@ def test_validation_without_gpu(L):
     assert L.diffattn_bwd_tc_workspace_size(2, 300, 3, 128) == up(4 * 600 * 3 * 2 * 256) + up(2 * 600 * 3 * 256) + \
         up(16 * 2 * 3 * 384)
     assert L.diffattn_bwd_tc_workspace_size(1, 0, 2, 64) == 0
+    # training pair
+    ft = lambda x, d, ws, wsb, mode=0: L.diffattn_fwd_train(x, x, x, x, 1, 16, 2, d, 1, x, 0.5, x, 1e-5, mode, ws, wsb,
+                                                            nul)
+    assert ft(fake, 96, fake, 1 << 30) == api.ERR_UNSUPPORTED
+    assert ft(fake, 128, nul, 1 << 30) == api.ERR_WORKSPACE
+    assert ft(fake, 128, fake, 16) == api.ERR_WORKSPACE
+    assert ft(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG
+    assert ft(fake, 128, fake, 1 << 30, mode=3) == api.ERR_INVALID_ARG
+    ts = lambda x, d, ws, wsb: L.diffattn_bwd_tc_saved(x, x, x, x, 1, 16, 2, d, 1, x, 0.5, x, 1e-5, 0,
+                                                       x, x, x, x, x, ws, wsb, nul)
+    assert ts(fake, 96, fake, 1 << 30) == api.ERR_UNSUPPORTED
+    assert ts(fake, 128, fake, 16) == api.ERR_WORKSPACE
+    assert ts(nul, 128, fake, 1 << 30) == api.ERR_INVALID_ARG
     # projections: sizes, multiples, pointers
     assert L.diffattn_rope_table(0, 64, 1e4, fake, nul) == api.ERR_INVALID_ARG
     assert L.diffattn_rope_table(16, 7, 1e4, fake, nul) == api.ERR_INVALID_ARG

@@ -156,3 +156,30 @@ def test_bwd_tc_rejects():
         api.diffattn_bwd_tc(inp.q, inp.k, inp.v, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, True,
                             workspace=small)
     assert e.value.status == api.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("B,N,H,d,causal,mode", [(1, 300, 2, 128, True, api.MODE_DIFF), (2, 130, 3, 64, False, api.MODE_SUM),
+                                                  (1, 517, 2, 128, True, api.MODE_LAMBDA_ZERO)])
+def test_train_forward_and_saved_backward(B, N, H, d, causal, mode):
+    """The training pair equals the separate calls: diffattn_fwd_train's output is bitwise the forward's,
+    and diffattn_bwd_tc_saved (statistics from the training forward) bitwise the backward that
+    recomputes them (dq, dk, dv; dlambda and dw are atomic sums, equal up to the order of the additions)."""
+    inp = wl.make_prefill(B, N, H, d, causal=causal, dtype="bf16", lambda_init=0.5, w="normal", seed=N + d,
+                          device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(11)
+    dy = torch.randn(inp.v.shape, generator=g, device="cuda").to(torch.bfloat16)
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+    y_ref = api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, causal, mode=mode)
+    y, ws = api.diffattn_fwd_train(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, causal, mode)
+    saved = api.diffattn_bwd_tc_saved(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, causal, mode,
+                                      ws)
+    fresh = api.diffattn_bwd_tc(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, causal, mode)
+    torch.cuda.synchronize()
+    assert api.device_status() == api.OK
+    assert torch.equal(y, y_ref)
+    for a, b in zip(saved[:3], fresh[:3]):
+        assert torch.equal(a, b)
+    # dlambda and dw add per-CTA partial sums with float atomics in the order the CTAs finish: reordering
+    # changes a sum of a few hundred fp32 partials by at most a few hundred roundings of the largest one
+    for a, b in zip(saved[3:], fresh[3:]):
+        assert (a - b).abs().max() <= 1e-4 * max(1.0, float(b.abs().max()))

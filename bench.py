@@ -461,7 +461,8 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{args.workload}: float64 CPU oracle, {rows} query rows of one head per step"},
+        "config": prefill_config(inp, args.workload, args.gpus, prefill_flops(*inp.q.shape[:3], d, inp.causal, "metric"),
+                                 prefill_flops(*inp.q.shape[:3], d, inp.causal, "algorithmic")),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"{rows} query rows per step (each against all {N} keys) of one seeded "
                                    f"(batch, head) of {args.workload}"},
@@ -470,6 +471,20 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def prefill_config(inp, name, world, flops_metric, flops_alg):
+    """The `config` object of the prefill line: the same for both arms."""
+    B, N, H, _, d = inp.q.shape
+    return {
+        "workload": f"{name}: B={B} N={N} H={H} d={d} V width {2 * d} "
+                    f"{'causal' if inp.causal else 'no mask'} bf16, per rank",
+        "flops_per_step_metric": flops_metric, "flops_per_step_algorithmic": flops_alg,
+        "flop_convention": "value: 16*N^2*d per head (half for causal), as the metric states; "
+                           "roofline: algorithmic 12*N^2*d per head (half for causal)",
+        "l2": f"inputs larger than L2: q+k+v = {3 * inp.q.numel() * 2 / 1e6:.0f} MB per step > 126 MB",
+        "parallelism": f"replicas x{world} (one process per GPU, no collective on the path)",
+    }
 
 
 # --------------------------------------------------------------------- ours --
@@ -618,15 +633,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {
-            "workload": f"{args.workload}: B={B} N={N} H={H} d={d} V width {2 * d} "
-                        f"{'causal' if inp.causal else 'no mask'} bf16, per rank",
-            "flops_per_step_metric": flops_metric, "flops_per_step_algorithmic": flops_alg,
-            "flop_convention": "value: 16*N^2*d per head (half for causal), as the metric states; "
-                               "roofline: algorithmic 12*N^2*d per head (half for causal)",
-            "l2": f"inputs larger than L2: q+k+v = {3 * inp.q.numel() * 2 / 1e6:.0f} MB per step > 126 MB",
-            "parallelism": f"replicas x{world} (one process per GPU, no collective on the path)",
-        },
+        "config": prefill_config(inp, args.workload, world, flops_metric, flops_alg),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "prefill_sm100_kernel<128>", "kernel_ms": kern_ms,

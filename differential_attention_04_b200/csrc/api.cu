@@ -119,7 +119,8 @@ int bwd_tc_impl(const void* q, const void* k, const void* v, const void* dy, int
   if (!encode_4d(&m.q128, q, d, 2ull * H, N, B) || !encode_4d(&m.q32, q, d, 2ull * H, N, B, 2, 32) ||
       !encode_4d(&m.k128, k, d, 2ull * H, N, B) || !encode_4d(&m.k32, k, d, 2ull * H, N, B, 2, 32) ||
       !encode_4d(&m.v128, v, 2ull * d, H, N, B) || !encode_4d(&m.v32, v, 2ull * d, H, N, B, 2, 32) ||
-      !encode_4d(&m.g128, g, 2ull * d, H, N, B) || !encode_4d(&m.g32, g, 2ull * d, H, N, B, 2, 32))
+      !encode_4d(&m.g128, g, 2ull * d, H, N, B) || !encode_4d(&m.g32, g, 2ull * d, H, N, B, 2, 32) ||
+      !encode_4d(&m.q64, q, d, 2ull * H, N, B, 2, 64) || !encode_4d(&m.g64, g, 2ull * d, H, N, B, 2, 64))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;

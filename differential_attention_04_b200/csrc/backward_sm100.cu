@@ -44,7 +44,6 @@ namespace {
 
 constexpr int kGradThreads = 256;
 constexpr int kRowTile = 128;  // rows of a gradient block (keys for dK and dV, queries for dQ)
-constexpr int kColTile = 32;   // streamed columns per tile
 constexpr float kLog2eBwd = 1.4426950408889634f;
 
 enum : int { kGradV = 0, kGradK = 1, kGradQ = 2 };
@@ -57,15 +56,20 @@ struct GCfg {
   static constexpr int QKB = D / 64;               // 128-byte boxes per Q / K row
   static constexpr int VGB = DV / 64;              // 128-byte boxes per V / G row
   static constexpr int RBOX = kRowTile * 128;      // [128 rows][128 bytes]
-  static constexpr int CBOX = kColTile * 128;      // [32 rows][128 bytes]
+  // Streamed columns per tile: 64 for dV (one S buffer; its S products are N = 64
+  // instructions, half as many as at N = 32 for the same columns), 32 for dK and
+  // dQ (two S buffers: S, dP and dS of two tiles share the 256 free columns).
+  static constexpr int NC = HAS_DP ? 32 : 64;
+  static constexpr int NSB = HAS_DP ? 2 : 1;  // S buffers in tensor memory
+  static constexpr int CBOX = NC * 128;       // [NC rows][128 bytes]
   // resident rows: both maps' K (dV, dK) or Q (dQ), then V (dK) or G (dQ)
   static constexpr int R_QK = 2 * QKB * RBOX;
   static constexpr int R_BYTES = R_QK + (HAS_DP ? VGB * RBOX : 0);
   // one column stage: both maps' Q (dV, dK) or K (dQ), then G (dV, dK) or V (dQ)
   static constexpr int C_QK = 2 * QKB * CBOX;
   static constexpr int C_BYTES = C_QK + VGB * CBOX;
-  static constexpr int ST_BYTES = kColTile * 16;  // one float4 of statistics per column
-  static constexpr int STAGES = HAS_DP ? 3 : 4;
+  static constexpr int ST_BYTES = NC * 16;  // one float4 of statistics per column
+  static constexpr int STAGES = HAS_DP ? 3 : 2;
   static constexpr int OFF_R = 0;
   static constexpr int OFF_C = R_BYTES;
   static constexpr int OFF_ST = OFF_C + STAGES * C_BYTES;
@@ -76,19 +80,26 @@ struct GCfg {
   static constexpr int SMEM_ALLOC = (SMEM_USED + 1024 > 116 * 1024) ? SMEM_USED + 1024 : 116 * 1024;
   // tensor memory: the accumulator, then two tile buffers of 128 columns
   static constexpr uint32_t TM_ACC = 0;  // dV (2d columns) or both maps' dK / dQ (d columns each)
+  // dK, dQ: two buffers of 128 columns at TM_BUF + 128 b: S_1 | S_2 | dP (float32,
+  // 32 columns each) | dS_1 | dS_2 (bf16 pairs, 16 columns each).
+  // dV: one S buffer at TM_BUF: S_1 | S_2 (64 columns each); two P buffers of 32
+  // columns (bf16 pairs) at TM_BUF + 128 + 32 b.
   static constexpr uint32_t TM_BUF = 256;
-  static constexpr uint32_t B_S1 = 0, B_S2 = 32, B_DP = 64;  // float32 [128 lanes][32 columns]
-  static constexpr uint32_t B_A1 = 96, B_A2 = 112;           // bf16 pairs [128 lanes][16 columns]
+  static constexpr uint32_t B_S1 = 0, B_S2 = NC, B_DP = 64;
+  static constexpr uint32_t B_A1 = 96, B_A2 = 112;
+  __device__ static uint32_t s_buf(int t) { return TM_BUF + (NSB == 2 ? 128u * (t & 1) : 0u); }
+  __device__ static uint32_t a_buf(int t) { return NSB == 2 ? s_buf(t) + B_A1 : TM_BUF + 2 * NC + (NC / 2) * (t & 1); }
   static constexpr uint32_t TM_COLS = 512;
   static_assert(R_BYTES % 1024 == 0 && C_BYTES % 1024 == 0, "operand tiles keep 1024-byte alignment");
+  static_assert(HAS_DP || TM_BUF + 2 * NC + NC <= 512, "dV's tensor memory: dV, one S buffer, two P buffers");
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
 struct GradBars {
   uint64_t r_full;  // the resident rows have landed
   uint64_t c_full[4], c_empty[4];
-  uint64_t s_full[2];  // S (and dP) of the tile in buffer b are in tensor memory
-  uint64_t s_free[2];  // the softmax warps have read them
+  uint64_t s_full[2];  // S (and dP) of the tile in S buffer b are in tensor memory
+  uint64_t s_free[2];  // the softmax warps have read them (dV: buffer 0 only)
   uint64_t a_full[2];  // P or dS of the tile is in tensor memory (bf16)
   uint64_t acc_done;   // the last gradient product has completed
   uint32_t tmem_base;
@@ -105,13 +116,6 @@ struct GradParams {
   int* status;
   unsigned long long limit_ns;
 };
-
-// Wait for every tcgen05.ld issued so far and pin 96 registers behind the wait.
-__device__ __forceinline__ void tmem_ld_wait3(uint32_t (&a)[32], uint32_t (&b)[32], uint32_t (&c)[32]) {
-  tmem_ld_wait(a);
-  tmem_ld_wait(b);
-  tmem_ld_wait(c);
-}
 
 template <int D, int KIND>
 __global__ void __launch_bounds__(kGradThreads, 1)
@@ -135,12 +139,14 @@ __global__ void __launch_bounds__(kGradThreads, 1)
   const int rt = (KIND == kGradQ) ? p.n_rtiles - 1 - li : li;
   const int b = bh / p.H, h = bh % p.H;
   const int row0 = rt * kRowTile;
-  int c_begin = 0, c_end = p.n_ctiles;
+  constexpr int NC = C::NC;
+  const int n_ctiles = (N + NC - 1) / NC;
+  int c_begin = 0, c_end = n_ctiles;
   if (p.causal) {
     if (KIND == kGradQ)
-      c_end = min(p.n_ctiles, (row0 + kRowTile) / kColTile);  // keys <= the block's last query
+      c_end = min(n_ctiles, (row0 + kRowTile) / NC);  // keys <= the block's last query
     else
-      c_begin = row0 / kColTile;  // queries >= the block's first key
+      c_begin = row0 / NC;  // queries >= the block's first key
   }
   const int T = c_end - c_begin;  // >= 1: row0 < N
 
@@ -195,7 +201,7 @@ __global__ void __launch_bounds__(kGradThreads, 1)
       for (; t < T; ++t) {
         const int st = t % C::STAGES;
         if (!mbar_wait(&bars->c_empty[st], ((t / C::STAGES) & 1) ^ 1, wc)) break;
-        const int c0 = (c_begin + t) * kColTile;
+        const int c0 = (c_begin + t) * NC;
         mbar_arrive_expect_tx(&bars->c_full[st], C::C_BYTES + (C::COL_STATS ? C::ST_BYTES : 0));
         uint8_t* base = sC + st * C::C_BYTES;
 #pragma unroll
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kGradThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kColTile, false, false);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, NC, false, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, KIND == kGradV ? C::DV : D, false, true);
       const uint32_t sRa = smem_u32(sR), sCa = smem_u32(sC);
       // Descriptors are built once and advanced by adding (offset >> 4) to
@@ -235,11 +241,16 @@ __global__ void __launch_bounds__(kGradThreads, 1)
       // tile i - 1's scores into P or dS.
       for (int i = 0; ok && i <= T; ++i) {
         if (i < T) {
-          const int bb = i & 1, st = i % C::STAGES;
-          if (i >= 2 && !(ok = mbar_wait(&bars->s_free[bb], ((i - 2) >> 1) & 1, wc))) break;
+          const int bb = (C::NSB == 2) ? (i & 1) : 0, st = i % C::STAGES;
+          // S_i overwrites the scores of tile i - NSB: the softmax warps must have read them
+          if (i >= C::NSB) {
+            const int jj = i - C::NSB;
+            const uint32_t ph = (C::NSB == 2) ? ((jj >> 1) & 1) : (jj & 1);
+            if (!(ok = mbar_wait(&bars->s_free[bb], ph, wc))) break;
+          }
           if (!(ok = mbar_wait(&bars->c_full[st], (i / C::STAGES) & 1, wc))) break;
           tc_fence_after();
-          const uint32_t tb = tmem + C::TM_BUF + 128u * bb;
+          const uint32_t tb = tmem + C::s_buf(i);
           const uint64_t cd = adv(c_desc, st * C::C_BYTES);
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
@@ -264,20 +275,19 @@ __global__ void __launch_bounds__(kGradThreads, 1)
           const int j = i - 1, bj = j & 1, stj = j % C::STAGES;
           if (!(ok = mbar_wait(&bars->a_full[bj], (j >> 1) & 1, wc))) break;
           tc_fence_after();
-          const uint32_t tb = tmem + C::TM_BUF + 128u * bj;
+          const uint32_t ta = tmem + C::a_buf(j);
           const uint64_t cd = adv(c_desc_mn, stj * C::C_BYTES);
           // B operands: the stage's rows [32][width] read MN-major (K = the 32 columns)
           if constexpr (KIND == kGradV) {
 #pragma unroll
-            for (int kk = 0; kk < kColTile / 16; ++kk)
-              umma_ts(tmem + C::TM_ACC, tb + C::B_A1 + 8 * kk, adv(cd, C::C_QK + kk * 2048), idesc_g,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < NC / 16; ++kk)
+              umma_ts(tmem + C::TM_ACC, ta + 8 * kk, adv(cd, C::C_QK + kk * 2048), idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
 #pragma unroll
-              for (int kk = 0; kk < kColTile / 16; ++kk)
-                umma_ts(tmem + C::TM_ACC + m * D, tb + (m ? C::B_A2 : C::B_A1) + 8 * kk,
+              for (int kk = 0; kk < NC / 16; ++kk)
+                umma_ts(tmem + C::TM_ACC + m * D, ta + (m ? C::B_A2 - C::B_A1 : 0u) + 8 * kk,
                         adv(cd, m * C::QKB * C::CBOX + kk * 2048), idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
@@ -301,38 +311,44 @@ __global__ void __launch_bounds__(kGradThreads, 1)
     const float4* stv = reinterpret_cast<const float4*>(sST);
     bool ok = true;
     for (int t = 0; t < T; ++t) {
-      const int bb = t & 1, st = t % C::STAGES;
-      if (!(ok = mbar_wait(&bars->s_full[bb], (t >> 1) & 1, wc))) break;
+      const int st = t % C::STAGES;
+      const int sb = (C::NSB == 2) ? (t & 1) : 0;
+      const uint32_t sph = (C::NSB == 2) ? ((t >> 1) & 1) : (t & 1);
+      if (!(ok = mbar_wait(&bars->s_full[sb], sph, wc))) break;
       if constexpr (C::COL_STATS) {  // the stage's statistics (bulk copy) are visible after this wait
         if (!(ok = mbar_wait(&bars->c_full[st], (t / C::STAGES) & 1, wc))) break;
       }
       tc_fence_after();
-      const uint32_t tb = tl + C::TM_BUF + 128u * bb;
-      uint32_t s1[32], s2[32], dp[32];
-      tmem_ld32(tb + C::B_S1, s1);
-      tmem_ld32(tb + C::B_S2, s2);
-      if constexpr (C::HAS_DP) {
-        tmem_ld32(tb + C::B_DP, dp);
-      } else {
+      const uint32_t tb = tl + C::s_buf(t);
+      uint32_t s1[NC], s2[NC], dp[C::HAS_DP ? NC : 1];
+      auto chunk = [](uint32_t* a, int h) -> uint32_t(&)[32] { return *reinterpret_cast<uint32_t(*)[32]>(a + 32 * h); };
 #pragma unroll
-        for (int c = 0; c < 32; ++c) dp[c] = 0u;
+      for (int h = 0; h < NC / 32; ++h) {
+        tmem_ld32(tb + C::B_S1 + 32 * h, chunk(s1, h));
+        tmem_ld32(tb + C::B_S2 + 32 * h, chunk(s2, h));
+        if constexpr (C::HAS_DP) tmem_ld32(tb + C::B_DP + 32 * h, chunk(dp, h));
       }
-      tmem_ld_wait3(s1, s2, dp);
+#pragma unroll
+      for (int h = 0; h < NC / 32; ++h) {  // one wait; these only order the registers behind it
+        tmem_ld_wait(chunk(s1, h));
+        tmem_ld_wait(chunk(s2, h));
+        if constexpr (C::HAS_DP) tmem_ld_wait(chunk(dp, h));
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[bb]);
+      if (lane == 0) mbar_arrive(&bars->s_free[sb]);
 
-      const int c0 = (c_begin + t) * kColTile;
-      bool masked = c0 + kColTile > N;
-      if (p.causal) masked = masked || (KIND == kGradQ ? (c0 + kColTile - 1 > row0) : (c0 < row0 + kRowTile - 1));
-      uint32_t a1[16], a2[16];
+      const int c0 = (c_begin + t) * NC;
+      bool masked = c0 + NC > N;
+      if (p.causal) masked = masked || (KIND == kGradQ ? (c0 + NC - 1 > row0) : (c0 < row0 + kRowTile - 1));
+      uint32_t a1[NC / 2], a2[NC / 2];
 #pragma unroll
-      for (int c2 = 0; c2 < 16; ++c2) {
+      for (int c2 = 0; c2 < NC / 2; ++c2) {
         float v1[2], v2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int c = 2 * c2 + e;
-          const float4 sv = C::COL_STATS ? stv[st * kColTile + c] : rs;
+          const float4 sv = C::COL_STATS ? stv[st * NC + c] : rs;
           const float p1 = fast_exp2(fmaf(__uint_as_float(s1[c]), sc, -sv.x));
           const float p2 = fast_exp2(fmaf(__uint_as_float(s2[c]), sc, -sv.y));
           if constexpr (KIND == kGradV) {
@@ -352,12 +368,19 @@ __global__ void __launch_bounds__(kGradThreads, 1)
         a1[c2] = pack_bf16x2(v1[0], v1[1]);
         if constexpr (KIND != kGradV) a2[c2] = pack_bf16x2(v2[0], v2[1]);
       }
-      tmem_st16(tb + C::B_A1, a1);
-      if constexpr (KIND != kGradV) tmem_st16(tb + C::B_A2, a2);
+      // P / dS buffer t & 1 was last read by the gradient product of tile t - 2,
+      // issued before S_t: the s_full wait above covers its completion
+      const uint32_t ta = tl + C::a_buf(t);
+      if constexpr (NC == 64) {
+        tmem_st32(ta, a1);
+      } else {
+        tmem_st16(ta, a1);
+        if constexpr (KIND != kGradV) tmem_st16(ta + (C::B_A2 - C::B_A1), a2);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->a_full[bb]);
+      if (lane == 0) mbar_arrive(&bars->a_full[t & 1]);
     }
 
     // ------------------------------------------------------- epilogue --
@@ -545,7 +568,7 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   prm.H = H;
   prm.causal = causal ? 1 : 0;
   prm.n_rtiles = (N + kRowTile - 1) / kRowTile;
-  prm.n_ctiles = (N + kColTile - 1) / kColTile;
+  prm.n_ctiles = 0;  // per kernel, from its column tile
   prm.n_pad = L.n_pad;
   prm.lambda = lambda;
   prm.mode = mode;
@@ -553,7 +576,7 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   prm.status = ctl.status;
   prm.limit_ns = ctl.limit_ns;
   prm.out = dv;
-  e = launch_grad<D, kGradV>(m.k128, m.k128, m.q32, m.g32, prm, stream);
+  e = launch_grad<D, kGradV>(m.k128, m.k128, m.q64, m.g64, prm, stream);
   if (e != cudaSuccess) return e;
   prm.out = dk;
   e = launch_grad<D, kGradK>(m.k128, m.v128, m.q32, m.g32, prm, stream);

@@ -50,9 +50,11 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
                        cudaStream_t stream);
 // Tensor-core backward (bf16 inputs, d in {64, 128}).  Maps over q, k
 // [B, N, H*2, d] and v, G [B, N, H, 2d] with boxes of 128 bytes x 128 rows
-// (q128 ...) or x 32 rows (q32 ...); G is the workspace's bf16 dO.
+// (q128 ...), x 64 rows (q64, g64) or x 32 rows (q32 ...); G is the
+// workspace's bf16 dO.
 struct BwdTcMaps {
   CUtensorMap q128, q32, k128, k32, v128, v32, g128, g32;
+  CUtensorMap q64, g64;  // the dV kernel's 64-row column tiles
 };
 // Workspace: per map A_i V as float32 [B, N, H, 2, 2d]; G bf16 [B, N, H, 2d];
 // statistics float4 [B][H][n_pad] (n_pad = N rounded up to 128).

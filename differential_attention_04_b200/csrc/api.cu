@@ -82,8 +82,8 @@ bool fits_i32(long long x) { return x >= 0 && x < (1ll << 31); }
 
 // A projection GEMM through launch_proj_gemm, with the maps over A [M, K] and B [n_total, K].
 int proj_launch(const void* a, const void* b, int M, int K, int n_total, ProjParams& prm, cudaStream_t stream) {
-  CUtensorMap ta, tb;
-  if (!encode_4d(&ta, a, K, 1, M, 1, 2, 128) || !encode_4d(&tb, b, K, 1, n_total, 1, 2, 256)) return DIFFATTN_ERR_CUDA;
+  CUtensorMap ta, tb;  // 2-SM tiles: each CTA of a pair loads 128 rows of A and 128 rows of B
+  if (!encode_4d(&ta, a, K, 1, M, 1, 2, 128) || !encode_4d(&tb, b, K, 1, n_total, 1, 2, 128)) return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
   prm.M = M;

@@ -80,13 +80,13 @@ cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* l
                               const float* dlambda, float* dlq1, float* dlk1, float* dlq2, float* dlk2,
                               cudaStream_t stream);
 
-// Projection GEMM C[M, N] = A[M, K] B[N, K]^T (bf16, fp32 accumulation, bf16
-// out; K a multiple of 64, N and the column boundaries multiples of 32).
-// Columns [col_end[o-1], col_end[o]) go to out[o] (row stride = that width);
-// columns below rope_end get RoPE from `rope` (float2 cos/sin [seq_len][d/2])
-// at position (row mod seq_len) when rope is non-null.  ta maps A as
-// (K, 1, M, 1) with boxes of 64 x 128 rows, tb maps B as (K, 1, N, 1) with
-// boxes of 64 x 256 rows.
+// Projection GEMM C[M, N] = A[M, K] B[N, K]^T on CTA pairs (tcgen05
+// cta_group::2; bf16, fp32 accumulation, bf16 out; K a multiple of 64, N and
+// the column boundaries multiples of 32).  Columns [col_end[o-1], col_end[o])
+// go to out[o] (row stride = that width); columns below rope_end get RoPE from
+// `rope` (float2 cos/sin [seq_len][d/2]) at position (row mod seq_len) when
+// rope is non-null.  ta maps A as (K, 1, M, 1), tb maps B as (K, 1, N, 1),
+// both with boxes of 64 x 128 rows.
 struct ProjParams {
   int M, N, K, seq_len, d, rope_end;
   int col_end[3];

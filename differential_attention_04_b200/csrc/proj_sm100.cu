@@ -7,18 +7,20 @@
 // "Differential Transformer", "Builds on"): consecutive channel pairs of each
 // d-wide Q1, Q2, K1, K2 rotated by n * base^(-2j/d) at token position n.
 //
-// One persistent GEMM kernel, C[M, N] = A[M, K] B[N, K]^T (bf16 operands,
-// fp32 accumulation in tensor memory, bf16 output):
-//   warp 0       TMA producer: A [128 x 64] and B [256 x 64] tiles, 4 stages
-//   warp 1       MMA issuer: tcgen05.mma M=128 N=256 K=16, two accumulator
-//                buffers of 256 columns so that a tile's epilogue overlaps
-//                the next tile's products
-//   warps 4-7    epilogue: one output row per thread, 32 columns at a time:
-//                rotate pairs (columns below rope_end) with the cos/sin
+// One persistent GEMM kernel on CTA pairs, C[M, N] = A[M, K] B[N, K]^T (bf16
+// operands, fp32 accumulation in tensor memory, bf16 output):
+//   warp 0       TMA producer (each CTA): its 128 rows of A and 128 rows of B
+//                per 64-wide K step, 6 stages
+//   warp 1       MMA issuer (the pair's leader): tcgen05.mma cta_group::2,
+//                M=256 N=256 K=16; two accumulator buffers of 256 columns in
+//                each CTA so that a tile's epilogue overlaps the next tile's
+//                products
+//   warps 4-7    epilogue (each CTA): one output row per thread, 32 columns at
+//                a time: rotate pairs (columns below rope_end) with the cos/sin
 //                table, round to bf16, store into the destination that owns
 //                the columns (q | k | v for the projection)
-// Tiles are visited in groups of 16 row blocks so that the CTAs working at
-// the same time share their B (weight) columns and A rows in L2.
+// Tiles are visited in groups of 8 row blocks (2048 rows) so that the pairs
+// working at the same time share their B (weight) columns and A rows in L2.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -30,51 +32,65 @@ namespace diffattn {
 namespace {
 
 constexpr int kPThreads = 256;
-constexpr int kPBM = 128, kPBN = 256, kPBK = 64;
-constexpr int kPStages = 4;
-constexpr int kPGroupM = 16;
-constexpr int kPABytes = kPBM * kPBK * 2;  // 16 KB
-constexpr int kPBBytes = kPBN * kPBK * 2;  // 32 KB
-constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPOffBar = kPStages * kPStageBytes;
-constexpr int kPSmem = kPOffBar + 256 + 1024;
-static_assert(kPSmem <= 232448, "shared memory per CTA");
+constexpr int kPBK = 64;  // K per stage: one 128-byte swizzle row of bf16
 
-struct ProjBars {
-  uint64_t full[kPStages], empty[kPStages];
+// A 256 x 256 tile per CTA pair, tcgen05.mma with cta_group::2 (M = 256)
+// issued by the pair's leader.  Each CTA loads its own 128 rows of A and its
+// own 128 rows of B (half the tile's N) per stage, so each SM's shared memory
+// carries half the B traffic of a one-CTA 128 x 256 tile; each CTA's tensor
+// memory receives its 128 rows of D.  Stage barriers live in the leader
+// (armed with both CTAs' bytes); the leader's commits arrive on both CTAs'
+// barriers; the peer's epilogue hands accumulators back to the leader with
+// remote arrivals.
+constexpr int k2BM = 256, k2BN = 256;
+constexpr int k2Stages = 6;
+constexpr int k2ABytes = 128 * kPBK * 2;  // this CTA's 128 rows of A
+constexpr int k2BBytes = 128 * kPBK * 2;  // this CTA's 128 rows of B
+constexpr int k2StageBytes = k2ABytes + k2BBytes;
+constexpr int k2OffBar = k2Stages * k2StageBytes;
+constexpr int k2Smem = k2OffBar + 256 + 1024;
+constexpr int k2GroupM = 8;
+static_assert(k2Smem <= 232448, "shared memory per CTA");
+
+struct Proj2Bars {
+  uint64_t full[k2Stages], empty[k2Stages];
   uint64_t acc_full[2], acc_empty[2];
-  uint64_t mma_done;  // every product this CTA issued has completed
+  uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
 };
 
 __global__ void __launch_bounds__(kPThreads, 1)
     proj_gemm_sm100_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
-                           const ProjParams p) {
+                         const ProjParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  ProjBars* bars = reinterpret_cast<ProjBars*>(smem + kPOffBar);
+  Proj2Bars* bars = reinterpret_cast<Proj2Bars*>(smem + k2OffBar);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tiles_m = (p.M + kPBM - 1) / kPBM, tiles_n = (p.N + kPBN - 1) / kPBN;
+  const uint32_t rank = cluster_ctarank();  // 0: the pair's leader (issues the MMAs)
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(blockIdx.x >> 1), n_cl = static_cast<int>(gridDim.x >> 1);
+  const int tiles_m = (p.M + k2BM - 1) / k2BM, tiles_n = (p.N + k2BN - 1) / k2BN;
   const int n_tiles = tiles_m * tiles_n;
   const int k_steps = p.K / kPBK;
   auto tile_coords = [&](int t, int& tm, int& tn) {
-    const int per_group = kPGroupM * tiles_n;
-    const int g = t / per_group, first = g * kPGroupM;
-    const int gm = min(kPGroupM, tiles_m - first);
+    const int per_group = k2GroupM * tiles_n;
+    const int g = t / per_group, first = g * k2GroupM;
+    const int gm = min(k2GroupM, tiles_m - first);
     const int r = t % per_group;
     tm = first + r % gm;
     tn = r / gm;
   };
+  auto lead = [&](uint64_t* bar) { return map_to_cta(smem_u32(bar), 0); };
 
   if (tid == 0) {
-    for (int i = 0; i < kPStages; ++i) {
+    for (int i = 0; i < k2Stages; ++i) {
       mbar_init(&bars->full[i], 1);
       mbar_init(&bars->empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->acc_full[i], 1);
-      mbar_init(&bars->acc_empty[i], 4);  // one arrival per epilogue warp
+      mbar_init(&bars->acc_empty[i], 8);  // every epilogue warp of both CTAs
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -85,11 +101,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
     tma_prefetch_desc(&tb);
   }
   if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(&bars->tmem_base, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const WaitCtl wc{p.status, &bars->abort, p.limit_ns};
@@ -99,52 +116,56 @@ __global__ void __launch_bounds__(kPThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
-      int it = 0;  // k steps issued (all tiles)
+      int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      for (int t = cid; ok && t < n_tiles; t += n_cl) {
         int tm, tn;
         tile_coords(t, tm, tn);
         for (int ks = 0; ks < k_steps; ++ks, ++it) {
-          const int s = it % kPStages;
-          if (!(ok = mbar_wait(&bars->empty[s], ((it / kPStages) & 1) ^ 1, wc))) break;
-          mbar_arrive_expect_tx(&bars->full[s], kPStageBytes);
-          uint8_t* st = smem + s * kPStageBytes;
-          tma_load_4d(st, &ta, &bars->full[s], ks * kPBK, 0, tm * kPBM, 0);
-          tma_load_4d(st + kPABytes, &tb, &bars->full[s], ks * kPBK, 0, tn * kPBN, 0);
+          const int s = it % k2Stages;
+          if (!(ok = mbar_wait(&bars->empty[s], ((it / k2Stages) & 1) ^ 1, wc))) break;
+          if (leader) mbar_arrive_expect_tx(&bars->full[s], 2 * k2StageBytes);
+          uint8_t* st = smem + s * k2StageBytes;
+          const uint32_t fb = lead(&bars->full[s]);
+          tma_load_4d_pair(st, &ta, fb, ks * kPBK, 0, tm * k2BM + 128 * static_cast<int>(rank), 0);
+          tma_load_4d_pair(st + k2ABytes, &tb, fb, ks * kPBK, 0, tn * k2BN + 128 * static_cast<int>(rank), 0);
         }
       }
-      for (int j = max(0, it - kPStages); j < it; ++j) mbar_wait(&bars->full[j % kPStages], (j / kPStages) & 1, wdrain);
+      // the leader's barriers count both CTAs' bytes: wait until nothing is still landing
+      if (leader)
+        for (int j = max(0, it - k2Stages); j < it; ++j)
+          mbar_wait(&bars->full[j % k2Stages], (j / k2Stages) & 1, wdrain);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kPBM, kPBN, false, false);
-      const uint32_t s0 = smem_u32(smem);
-      int it = 0, lt = 0;  // k steps consumed, tiles done (this CTA)
+    // ------------------------------------------------ MMA issuer (leader) --
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(k2BM, k2BN, false, false);
+      const uint64_t s_desc = smem_desc_sw128(smem_u32(smem), 16, 1024);
+      auto adv = [](uint64_t desc, uint32_t bytes) { return desc + static_cast<uint64_t>(bytes >> 4); };
+      int it = 0, lt = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
+      for (int t = cid; ok && t < n_tiles; t += n_cl, ++lt) {
         const int ab = lt & 1;
-        // the epilogue has drained this accumulator buffer (tile lt - 2)
-        if (lt >= 2 && !(ok = mbar_wait(&bars->acc_empty[ab], ((lt - 2) >> 1) & 1, wc))) break;
+        // both CTAs' epilogues have drained this accumulator buffer (tile lt - 2)
+        if (lt >= 2 && !(ok = mbar_wait_acq_cluster(&bars->acc_empty[ab], ((lt - 2) >> 1) & 1, wc))) break;
         tc_fence_after();
         for (int ks = 0; ks < k_steps; ++ks, ++it) {
-          const int s = it % kPStages;
-          if (!(ok = mbar_wait(&bars->full[s], (it / kPStages) & 1, wc))) break;
+          const int s = it % k2Stages;
+          if (!(ok = mbar_wait(&bars->full[s], (it / k2Stages) & 1, wc))) break;
           tc_fence_after();
-          const uint32_t sa = s0 + s * kPStageBytes, sb = sa + kPABytes;
+          const uint32_t so = s * k2StageBytes;
 #pragma unroll
           for (int kk = 0; kk < kPBK / 16; ++kk)
-            umma_ss(tmem + 256u * ab, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024),
-                    idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars->empty[s]);  // the stage is free once these products have read it
+            umma_ss_pair(tmem + 256u * ab, adv(s_desc, so + kk * 32), adv(s_desc, so + k2ABytes + kk * 32), idesc,
+                         (ks > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair_mc(&bars->empty[s], 0x3);  // both CTAs' stage s is free once these have read it
         }
-        if (ok) umma_commit(&bars->acc_full[ab]);
+        if (ok) umma_commit_pair_mc(&bars->acc_full[ab], 0x3);
       }
-      // drain: no product may still be writing tensor memory when it is freed
-      umma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0, wdrain);
+      umma_commit_pair_mc(&bars->mma_done, 0x3);  // drain: both CTAs learn when every product has completed
     }
+    if (lane == 0) mbar_wait(&bars->mma_done, 0, wdrain);
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue --
@@ -152,29 +173,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int r = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     int lt = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
+    for (int t = cid; t < n_tiles; t += n_cl, ++lt) {
       const int ab = lt & 1;
       int tm, tn;
       tile_coords(t, tm, tn);
       if (!mbar_wait(&bars->acc_full[ab], (lt >> 1) & 1, wc)) break;
       tc_fence_after();
-      const int m = tm * kPBM + r;
+      const int m = tm * k2BM + 128 * static_cast<int>(rank) + r;
       const bool live = m < p.M;
       const int pos = live ? m % p.seq_len : 0;
 #pragma unroll 1
-      for (int c = 0; c < kPBN / 32; ++c) {
+      for (int c = 0; c < k2BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32_sync(tl + 256u * ab + 32 * c, v);
-        const int col = tn * kPBN + 32 * c;
+        const int col = tn * k2BN + 32 * c;
         if (!live || col >= p.N) continue;
-        // destination: the output owning these 32 columns (selects, no indexed parameter reads)
         const bool in0 = col < p.col_end[0], in1 = !in0 && col < p.col_end[1];
         const int start = in0 ? 0 : (in1 ? p.col_end[0] : p.col_end[1]);
         const int width = (in0 ? p.col_end[0] : (in1 ? p.col_end[1] : p.col_end[2])) - start;
         __nv_bfloat16* obase = in0 ? p.out[0] : (in1 ? p.out[1] : p.out[2]);
         const int c_in = col - start;
         if (p.rope && col < p.rope_end) {
-          // rotate 16 consecutive pairs: channel (c_in mod d), position pos
           const float2* cs = p.rope + static_cast<size_t>(pos) * (p.d / 2) + (c_in % p.d) / 2;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -194,15 +213,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
+      if (lane == 0) mbar_arrive_remote(lead(&bars->acc_empty[ab]));  // this CTA's rows of the buffer are read
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no remote access to either CTA remains
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -220,21 +240,34 @@ __global__ void rope_table_kernel(int seq_len, int d, double base, float2* table
 }  // namespace
 
 cudaError_t launch_proj_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const ProjParams& prm,
-                             cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(proj_gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+                                 cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(proj_gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
   if (e != cudaSuccess) return e;
-  static int sms[64] = {};
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.dynamicSmemBytes = k2Smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (sms[dev] == 0) {
+  int& mc = max_clusters[dev];
+  if (mc == 0) {
+    cfg.gridDim = dim3(2 * 128, 1, 1);
     int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 1;
-    sms[dev] = n;
+    if (cudaOccupancyMaxActiveClusters(&n, proj_gemm_sm100_kernel, &cfg) != cudaSuccess || n < 1) n = 1;
+    mc = n;
   }
-  const int tiles = ((prm.M + kPBM - 1) / kPBM) * ((prm.N + kPBN - 1) / kPBN);
-  const int grid = tiles < sms[dev] ? tiles : sms[dev];
-  proj_gemm_sm100_kernel<<<grid, kPThreads, kPSmem, stream>>>(ta, tb, prm);
-  return cudaGetLastError();
+  const int tiles = ((prm.M + k2BM - 1) / k2BM) * ((prm.N + k2BN - 1) / k2BN);
+  const int clusters = tiles < mc ? tiles : mc;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  return cudaLaunchKernelEx(&cfg, proj_gemm_sm100_kernel, ta, tb, prm);
 }
 
 cudaError_t launch_rope_table(int seq_len, int d, double base, float* table, cudaStream_t stream) {

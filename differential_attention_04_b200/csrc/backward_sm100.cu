@@ -21,8 +21,8 @@
 //        dV  rows = keys:    S_i^T = K_i Q_i^T,  dV += (P_1 + c P_2)^T G
 //        dK  rows = keys:    S_i^T, dP^T = V G^T, dK_i += dS_i^T Q_i
 //        dQ  rows = queries: S_i, dP = G V^T,     dQ_i += dS_i K_i
-//      The row operands stay in shared memory; 32-column tiles of the other
-//      side stream through a TMA ring.  S (and dP) land in tensor memory;
+//      The row operands stay in shared memory; column tiles of the other side
+//      (32 columns for dK and dQ, 64 for dV) stream through a TMA ring.  S (and dP) land in tensor memory;
 //      four softmax warps turn them into P or dS, store them back into
 //      tensor memory as bf16, and the gradient product reads them from
 //      there as its A operand (tcgen05.mma with A in tensor memory).  The
@@ -108,7 +108,7 @@ struct GradBars {
 
 struct GradParams {
   int B, N, H, causal;
-  int n_rtiles, n_ctiles, n_pad;
+  int n_rtiles, n_pad;
   const float* lambda;
   int mode;
   const float4* stats;  // [B][H][n_pad]: lse_1, lse_2 (scaled log2 units), D_1, D_2
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kGradThreads, 1)
           tc_fence_after();
           const uint32_t ta = tmem + C::a_buf(j);
           const uint64_t cd = adv(c_desc_mn, stj * C::C_BYTES);
-          // B operands: the stage's rows [32][width] read MN-major (K = the 32 columns)
+          // B operands: the stage's rows [NC][width] read MN-major (K = the NC columns)
           if constexpr (KIND == kGradV) {
 #pragma unroll
             for (int kk = 0; kk < NC / 16; ++kk)
@@ -568,7 +568,6 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   prm.H = H;
   prm.causal = causal ? 1 : 0;
   prm.n_rtiles = (N + kRowTile - 1) / kRowTile;
-  prm.n_ctiles = 0;  // per kernel, from its column tile
   prm.n_pad = L.n_pad;
   prm.lambda = lambda;
   prm.mode = mode;

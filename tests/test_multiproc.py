@@ -72,3 +72,12 @@ def test_reference_arm_two_ranks_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the line keeps the contract's keys, and the GPU arm's metric and config
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "gpu_launches"):
+        assert key in d, key
+    assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["n_gpus"] == 2
+    assert d["config"]["workload"].startswith("prefill_3b: B=4 N=4096 H=12 d=128 V width 256 causal bf16")
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["cores"] >= 1
+    import bench
+    assert d["metric"] == bench.METRIC

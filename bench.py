@@ -50,6 +50,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-qk8", action="store_true")
+    ap.add_argument("--no-qk4", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--bwd-steps", type=int, default=50)
     ap.add_argument("--no-proj", action="store_true")
@@ -385,22 +386,26 @@ def bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, K):
             "gpu_launches": 2 * K}
 
 
-def bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K):
-    """The e4m3 query/key variant on the same workload: a step quantises q and k
-    (one absmax scale per batch, head and map) and runs the prefill whose
-    scores are 8-bit tensor-core products."""
+def bench_lowbit(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K, bits=8):
+    """The low-bit query/key variant on the same workload: a step quantises q
+    and k (one absmax scale per batch, head and map; e4m3 codes for bits=8,
+    packed e2m1 codes for bits=4) and runs the prefill whose scores are
+    kind::f8f6f4 tensor-core products of the codes."""
     import torch
 
     B, N, H, _, d = inp.q.shape
-    qc, qs = api.quantize_qk(inp.q)
-    kc, ks = api.quantize_qk(inp.k)
+    quantize = api.quantize_qk if bits == 8 else api.quantize_qk4
+    forward = api.diffattn_fwd_qk8 if bits == 8 else api.diffattn_fwd_qk4
+    fmt = "e4m3" if bits == 8 else "e2m1"
+    qc, qs = quantize(inp.q)
+    kc, ks = quantize(inp.k)
 
     def quant():
-        api.quantize_qk(inp.q, qc, qs)
-        api.quantize_qk(inp.k, kc, ks)
+        quantize(inp.q, qc, qs)
+        quantize(inp.k, kc, ks)
 
     def fwd():
-        api.diffattn_fwd_qk8(qc, qs, kc, ks, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
+        forward(qc, qs, kc, ks, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
 
     for _ in range(5):
         quant()
@@ -420,16 +425,17 @@ def bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K):
     flops_metric = prefill_flops(B, N, H, d, inp.causal, "metric")
     flops_alg = prefill_flops(B, N, H, d, inp.causal, "algorithmic")
     # a third of the algorithmic flops (the scores, 4d of 12d per pair) run on the
-    # 8-bit path at twice the bf16 rate: the mixed peak is 1 / (1/6 + 2/3) = 1.2 x bf16
+    # kind::f8f6f4 path at twice the bf16 rate (e4m3 and e2m1 operands alike; only the
+    # block-scaled fp4 kinds go faster): the mixed peak is 1 / (1/6 + 2/3) = 1.2 x bf16
     bf16_peak = peaks["bf16_tflops"]
     mixed = 1.2 * bf16_peak
     achieved = flops_alg / (f_ms * 1e-3) / 1e12
-    return {"metric": "DiffAttn fwd TFLOP/s, e4m3 queries/keys (quantise + prefill)",
+    return {"metric": f"DiffAttn fwd TFLOP/s, {fmt} queries/keys (quantise + prefill)",
             "value": flops_metric / ((q_ms + f_ms) * 1e-3) / 1e12, "unit": "TFLOP/s", "steps": K,
             "ms_per_step": q_ms + f_ms, "quantize_ms": q_ms, "prefill_ms": f_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": mixed, "unit": "TFLOP/s",
-                         "frac": achieved / mixed, "traffic": None, "kernel": "prefill_sm100_kernel<128, e4m3>",
-                         "peak_source": f"{peak_src} bf16 dense (burst) x 1.2: scores on the 8-bit path at the "
+                         "frac": achieved / mixed, "traffic": None, "kernel": f"prefill_sm100_kernel<128, {fmt}>",
+                         "peak_source": f"{peak_src} bf16 dense (burst) x 1.2: scores on the f8f6f4 path at the "
                                         "nominal 2x rate"},
             "gpu_launches": 7 * K}
 
@@ -653,7 +659,9 @@ def run_ours(args):
     if not args.no_proj:
         line["proj"] = bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, args.proj_steps)
     if not args.no_qk8 and d == 128:
-        line["qk8"] = bench_qk8(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8))
+        line["qk8"] = bench_lowbit(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8), 8)
+    if not args.no_qk4 and d == 128:
+        line["qk4"] = bench_lowbit(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8), 4)
     if not args.no_decode:
         line["decode"] = bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world)
     del inp, y

@@ -24,6 +24,9 @@ SIGNATURES = {
     "diffattn_quantize_qk": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "diffattn_fwd_qk8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                   _vp, _c_float, _vp, _c_float, _c_int, _vp]),
+    "diffattn_quantize_qk4": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "diffattn_fwd_qk4": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                  _vp, _c_float, _vp, _c_float, _c_int, _vp]),
     "diffattn_bwd_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "diffattn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_float,
                               _vp, _c_float, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),

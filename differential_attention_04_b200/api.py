@@ -131,6 +131,50 @@ def diffattn_fwd_qk8(q_codes: torch.Tensor, q_scales: torch.Tensor, k_codes: tor
     return out
 
 
+def quantize_qk4(x: torch.Tensor, codes: torch.Tensor | None = None,
+                 scales: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """e2m1 codes, two per byte (uint8 [B, N, H, 2, d / 2], channel 2j in the low nibble), and float32
+    scales [B, H, 2] of a bf16 q or k [B, N, H, 2, d]: one absmax scale per (batch, head, map)."""
+    _dev(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 5 or x.shape[3] != 2:
+        raise ValueError("x must be bfloat16 [B, N, H, 2, d]")
+    B, N, H, _, d = x.shape
+    if d % 8:
+        raise ValueError("d must be a multiple of 8")
+    shape = (B, N, H, 2, d // 2)
+    if codes is None:
+        codes = torch.empty(shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, 2), dtype=torch.float32, device=x.device)
+    _dev(codes, scales)
+    if tuple(codes.shape) != shape or codes.dtype != torch.uint8 or scales.numel() != B * H * 2 or \
+            scales.dtype != torch.float32:
+        raise ValueError("codes must be uint8 [B, N, H, 2, d / 2] and scales float32 [B, H, 2]")
+    _check("diffattn_quantize_qk4", lib().diffattn_quantize_qk4(_ptr(x), B, N, H, d, _ptr(codes), _ptr(scales),
+                                                                _stream()))
+    return codes, scales
+
+
+def diffattn_fwd_qk4(q_codes: torch.Tensor, q_scales: torch.Tensor, k_codes: torch.Tensor, k_scales: torch.Tensor,
+                     v: torch.Tensor, lam: torch.Tensor, lambda_init: float, rms_w: torch.Tensor, eps: float = 1e-5,
+                     causal: bool = True, out: torch.Tensor | None = None, mode: int = MODE_DIFF) -> torch.Tensor:
+    """Prefill with e2m1 queries and keys (as quantize_qk4 returns them, [B, N, H, 2, d / 2]);
+    v, out: bf16 [B, N, H, 2d]."""
+    _dev(q_codes, q_scales, k_codes, k_scales, v, lam, rms_w)
+    B, N, H, two, half = q_codes.shape
+    d = 2 * half
+    if q_codes.dtype != torch.uint8 or k_codes.dtype != torch.uint8 or k_codes.shape != q_codes.shape or two != 2:
+        raise ValueError("q_codes, k_codes must be uint8 [B, N, H, 2, d / 2]")
+    if v.dtype != torch.bfloat16 or tuple(v.shape) != (B, N, H, 2 * d):
+        raise ValueError("v must be bfloat16 [B, N, H, 2d]")
+    if out is None:
+        out = torch.empty_like(v)
+    _check("diffattn_fwd_qk4", lib().diffattn_fwd_qk4(
+        _ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v), _ptr(out), B, N, H, d,
+        int(bool(causal)), _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode), _stream()))
+    return out
+
+
 def bwd_workspace_size(B: int, N: int, H: int, d: int) -> int:
     return int(lib().diffattn_bwd_workspace_size(B, N, H, d))
 

@@ -78,7 +78,67 @@ bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D map over packed e2m1 codes, dims (innermost first) d0 codes (two per
+// byte; d0 a multiple of 128), d1..d3; box = 128 codes x 1 x 128 rows x 1,
+// widened to 128 bytes a row in shared memory (8 bytes of codes, then 8 bytes
+// of gap, per 16 codes), 128-byte swizzle, zero fill out of bounds.  The base
+// must be 32-byte aligned and every stride a multiple of 32 bytes.
+bool encode_4d_e2m1(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 / 2, d0 / 2 * d1, d0 / 2 * d1 * d2};
+  const cuuint32_t box[4] = {128, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool fits_i32(long long x) { return x >= 0 && x < (1ll << 31); }
+
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+int quantize_impl(const void* x, int B, int N, int H, int d, int bits, void* codes, float* scales,
+                  cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 1 || d < 8 || d % 8 != 0) return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (!x || !codes || !scales) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return DIFFATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * 2 > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  return cuda_status(launch_quantize_qk(x, B, N, H, d, bits, codes, scales, stream));
+}
+
+// The prefill on low-bit query and key codes: bits 8 (e4m3) or 4 (packed e2m1).
+int fwd_lowbit_impl(int bits, const void* q_codes, const float* q_scales, const void* k_codes,
+                    const float* k_scales, const void* v, void* o, int B, int N, int H, int d, int causal,
+                    const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
+                    cudaStream_t stream) {
+  if (B < 1 || H < 1 || N < 0 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
+  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
+  if (N == 0) return DIFFATTN_OK;
+  if (!q_codes || !q_scales || !k_codes || !k_scales || !v || !o || !lambda || !rms_w)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !aligned16(v) || !aligned16(o)) return DIFFATTN_ERR_INVALID_ARG;
+  if (bits == 4 && (!aligned32(q_codes) || !aligned32(k_codes))) return DIFFATTN_ERR_INVALID_ARG;
+  if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv, to;
+  const bool codes_ok = bits == 4 ? encode_4d_e2m1(&tq, q_codes, d, 2ull * H, N, B) &&
+                                        encode_4d_e2m1(&tk, k_codes, d, 2ull * H, N, B)
+                                  : encode_4d(&tq, q_codes, d, 2ull * H, N, B, 1) &&
+                                        encode_4d(&tk, k_codes, d, 2ull * H, N, B, 1);
+  if (!codes_ok || !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
+    return DIFFATTN_ERR_CUDA;
+  DevCtl ctl;
+  cudaError_t e = status_ptr(&ctl.status);
+  if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  ctl.limit_ns = g_wait_limit_ns.load();
+  return cuda_status(launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
+                                          mode, q_scales, k_scales, bits, ctl, stream));
+}
 
 // A projection GEMM through launch_proj_gemm, with the maps over A [M, K] and B [n_total, K].
 int proj_launch(const void* a, const void* b, int M, int K, int n_total, ProjParams& prm, cudaStream_t stream) {
@@ -209,42 +269,31 @@ int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o, int 
   ctl.limit_ns = g_wait_limit_ns.load();
   return cuda_status(
       launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, nullptr,
-                           nullptr, ctl, stream));
+                           nullptr, 16, ctl, stream));
 }
 
 int diffattn_quantize_qk(const void* x, int B, int N, int H, int d, void* codes, float* scales,
                          cudaStream_t stream) {
-  if (B < 1 || H < 1 || N < 1 || d < 8 || d % 8 != 0) return DIFFATTN_ERR_INVALID_ARG;
-  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
-  if (!x || !codes || !scales) return DIFFATTN_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return DIFFATTN_ERR_INVALID_ARG;
-  if (static_cast<long long>(B) * H * 2 > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  return cuda_status(launch_quantize_qk(x, B, N, H, d, codes, scales, stream));
+  return quantize_impl(x, B, N, H, d, 8, codes, scales, stream);
+}
+
+int diffattn_quantize_qk4(const void* x, int B, int N, int H, int d, void* codes, float* scales,
+                          cudaStream_t stream) {
+  return quantize_impl(x, B, N, H, d, 4, codes, scales, stream);
 }
 
 int diffattn_fwd_qk8(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,
                      const void* v, void* o, int B, int N, int H, int d, int causal, const float* lambda,
                      float lambda_init, const float* rms_w, float eps, int mode, cudaStream_t stream) {
-  if (B < 1 || H < 1 || N < 0 || d < 1 || !(eps >= 0.f)) return DIFFATTN_ERR_INVALID_ARG;
-  if (mode != DIFFATTN_MODE_DIFF && mode != DIFFATTN_MODE_LAMBDA_ZERO && mode != DIFFATTN_MODE_SUM)
-    return DIFFATTN_ERR_INVALID_ARG;
-  if (!fits_i32(static_cast<long long>(B) * N * H * 2 * d)) return DIFFATTN_ERR_INVALID_ARG;
-  if (N == 0) return DIFFATTN_OK;
-  if (!q_codes || !q_scales || !k_codes || !k_scales || !v || !o || !lambda || !rms_w)
-    return DIFFATTN_ERR_INVALID_ARG;
-  if (!aligned16(q_codes) || !aligned16(k_codes) || !aligned16(v) || !aligned16(o)) return DIFFATTN_ERR_INVALID_ARG;
-  if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
-  if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv, to;
-  if (!encode_4d(&tq, q_codes, d, 2ull * H, N, B, 1) || !encode_4d(&tk, k_codes, d, 2ull * H, N, B, 1) ||
-      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
-    return DIFFATTN_ERR_CUDA;
-  DevCtl ctl;
-  cudaError_t e = status_ptr(&ctl.status);
-  if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
-  ctl.limit_ns = g_wait_limit_ns.load();
-  return cuda_status(launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
-                                          mode, q_scales, k_scales, ctl, stream));
+  return fwd_lowbit_impl(8, q_codes, q_scales, k_codes, k_scales, v, o, B, N, H, d, causal, lambda, lambda_init,
+                         rms_w, eps, mode, stream);
+}
+
+int diffattn_fwd_qk4(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,
+                     const void* v, void* o, int B, int N, int H, int d, int causal, const float* lambda,
+                     float lambda_init, const float* rms_w, float eps, int mode, cudaStream_t stream) {
+  return fwd_lowbit_impl(4, q_codes, q_scales, k_codes, k_scales, v, o, B, N, H, d, causal, lambda, lambda_init,
+                         rms_w, eps, mode, stream);
 }
 
 size_t diffattn_bwd_workspace_size(int B, int N, int H, int d) {

@@ -277,12 +277,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          | (static_cast<uint32_t>(M >> 4) << 24); // M >> 4
 }
 
-// Instruction descriptor for kind::f8f6f4 with e4m3 A/B (both K-major) and
-// fp32 D; K = 32 per instruction.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+// Instruction descriptor for kind::f8f6f4 with A and B of one format (both
+// K-major) and fp32 D; K = 32 elements per instruction.  Format codes: e4m3 0,
+// e2m1 5 (e2m1 read from shared memory as 8 bytes of packed codes in every 16).
+constexpr uint32_t kF8f6f4E4m3 = 0;
+constexpr uint32_t kF8f6f4E2m1 = 5;
+__host__ __device__ constexpr uint32_t idesc_f8f6f4_f32(int M, int N, uint32_t ab_format) {
   return (1u << 4)                                // D format: f32
-         | (0u << 7)                              // A format: e4m3
-         | (0u << 10)                             // B format: e4m3
+         | (ab_format << 7)                       // A format
+         | (ab_format << 10)                      // B format
          | (static_cast<uint32_t>(N >> 3) << 17)  // N >> 3
          | (static_cast<uint32_t>(M >> 4) << 24); // M >> 4
 }

@@ -28,18 +28,21 @@ __host__ __device__ inline float map2_coefficient(int mode, float lam) {
 }
 
 // Tensor-core (tcgen05) prefill, d in {64, 128} for bf16 queries and keys,
-// d = 128 for e4m3 ones (q_scale, k_scale non-null).  tq/tk map
-// [B, N, H*2, d]; tv and to map [B, N, H, 2d]; boxes are 128 bytes x 128 rows
-// with 128-byte swizzle.
+// d = 128 for low-bit ones (q_scale, k_scale non-null; qk_bits 8: e4m3 codes,
+// 4: packed e2m1 codes).  tq/tk map [B, N, H*2, d]; tv and to map
+// [B, N, H, 2d]; boxes are 128 bytes (bf16, e4m3) or 128 elements (e2m1) x
+// 128 rows with 128-byte swizzle.
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, int mode, const float* q_scale,
-                                 const float* k_scale, DevCtl ctl, cudaStream_t stream);
+                                 const float* k_scale, int qk_bits, DevCtl ctl, cudaStream_t stream);
 
-// e4m3 codes of a bf16 [B, N, H, 2, d] tensor with one float32 scale per
+// Low-bit codes of a bf16 [B, N, H, 2, d] tensor with one float32 scale per
 // (batch, head, map) (scales: [B][H][2], also the absmax accumulator).
-cudaError_t launch_quantize_qk(const void* x, int B, int N, int H, int d, void* codes, float* scales,
+// bits 8: e4m3 codes, one byte each; bits 4: e2m1 codes, two per byte
+// (channel 2j in the low nibble).
+cudaError_t launch_quantize_qk(const void* x, int B, int N, int H, int d, int bits, void* codes, float* scales,
                                cudaStream_t stream);
 
 // Backward pass of the prefill (CUDA cores; bf16 or fp32 inputs, fp32 gradients).

@@ -71,9 +71,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kOverflowGuard = 64.0f;    // log2 units
 
-// QK8: queries and keys arrive as e4m3 codes (one byte each) with a float32
-// scale per (batch, head, map); S is then a kind::f8f6f4 product.  Otherwise
-// they are bf16 and S is a kind::f16 product.
+// QK8: queries and keys arrive as low-bit codes with a float32 scale per
+// (batch, head, map) and S is a kind::f8f6f4 product: e4m3 codes take one
+// byte each; e2m1 codes come packed two per byte and the tensor map
+// (16U4_ALIGN16B) widens every 8 bytes of them to 16 in shared memory, so both
+// formats leave one byte of shared memory per element.  Otherwise they are
+// bf16 and S is a kind::f16 product.
 template <int D, bool QK8>
 struct Cfg {
   static constexpr int DV = 2 * D;
@@ -156,12 +159,18 @@ __device__ __forceinline__ void tmem_ld_wait4(uint32_t (&a)[32], uint32_t (&b)[3
 // log-sum-exp (what the backward pass needs); kOutBoth both (a training
 // forward that saves the backward's statistics).
 enum : int { kOutNorm = 0, kOutStats = 1, kOutBoth = 2 };
-template <int D, bool QK8, int OUT>
+// QKF: the format of the queries and keys
+enum : int { kQkBf16 = 0, kQkE4m3 = 1, kQkE2m1 = 2 };
+template <int D, int QKF, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                          const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
                          const PrefillParams p) {
+  constexpr bool QK8 = QKF != kQkBf16;
   using C = Cfg<D, QK8>;
+  // bytes a Q / K tile brings in from global memory (packed e2m1: half its shared-memory size)
+  constexpr uint32_t kQTx = QKF == kQkE2m1 ? C::Q_BYTES / 2 : C::Q_BYTES;
+  constexpr uint32_t kKTx = QKF == kQkE2m1 ? C::K_BYTES / 2 : C::K_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -254,14 +263,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c1 = 2 * it.h + static_cast<int>(rank);
         // Q of this item replaces the last one's once that item's S products have read it
         if (k > 0 && !(ok = mbar_wait(&bars->q_empty, (k - 1) & 1, wc))) break;
-        mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+        mbar_arrive_expect_tx(&bars->q_full, kQTx);
 #pragma unroll
         for (int blk = 0; blk < C::QBLK; ++blk)
           tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * C::QBOX, c1, it.qtile * kBM, it.b);
         for (int j = 0; j < it.n_kv; ++j, ++gk) {
           const int st = gk & 1;
           if (!(ok = mbar_wait(&bars->k_empty[st], ((gk >> 1) & 1) ^ 1, wc))) break;
-          mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
+          mbar_arrive_expect_tx(&bars->k_full[st], kKTx);
 #pragma unroll
           for (int blk = 0; blk < C::QBLK; ++blk)
             tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * C::QBOX, c1,
@@ -299,7 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idesc_s = QK8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_s = QKF == kQkE2m1   ? idesc_f8f6f4_f32(128, 128, kF8f6f4E2m1)
+                                   : QKF == kQkE4m3 ? idesc_f8f6f4_f32(128, 128, kF8f6f4E4m3)
+                                                    : idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       int gs = 0;  // S products issued (all items)
@@ -631,11 +642,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool QK8, int OUT = kOutNorm>
+template <int D, int QKF, int OUT = kOutNorm>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const PrefillParams& prm, cudaStream_t stream) {
-  using C = Cfg<D, QK8>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QK8, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  using C = Cfg<D, QKF != kQkBf16>;
+  cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QKF, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -657,19 +668,19 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if (mc == 0) {
     cfg.gridDim = dim3(2 * 128, 1, 1);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QK8, OUT>, &cfg) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<D, QKF, OUT>, &cfg) != cudaSuccess || n < 1) n = 1;
     mc = n;
   }
   const int clusters = prm.n_items < mc ? prm.n_items : mc;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QK8, OUT>, tq, tk, tv, to, prm);
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QKF, OUT>, tq, tk, tv, to, prm);
 }
 
 cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, int mode, const float* q_scale,
-                                 const float* k_scale, DevCtl ctl, cudaStream_t stream) {
+                                 const float* k_scale, int qk_bits, DevCtl ctl, cudaStream_t stream) {
   PrefillParams prm = {};
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.N = N;
@@ -692,10 +703,14 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.eps = eps;
   prm.status = ctl.status;
   prm.limit_ns = ctl.limit_ns;
-  const bool qk8 = q_scale != nullptr;
-  if (qk8) return d == 128 ? launch_d<128, true>(tq, tk, tv, to, prm, stream) : cudaErrorInvalidValue;
-  if (d == 128) return launch_d<128, false>(tq, tk, tv, to, prm, stream);
-  if (d == 64) return launch_d<64, false>(tq, tk, tv, to, prm, stream);
+  if (q_scale != nullptr) {
+    if (d != 128) return cudaErrorInvalidValue;
+    if (qk_bits == 8) return launch_d<128, kQkE4m3>(tq, tk, tv, to, prm, stream);
+    if (qk_bits == 4) return launch_d<128, kQkE2m1>(tq, tk, tv, to, prm, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (d == 128) return launch_d<128, kQkBf16>(tq, tk, tv, to, prm, stream);
+  if (d == 64) return launch_d<64, kQkBf16>(tq, tk, tv, to, prm, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -727,13 +742,13 @@ cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap&
   prm.lse = lse;
   prm.n_pad = n_pad;
   if (to) {  // the normalised output as well
-    if (d == 128) return launch_d<128, false, kOutBoth>(tq, tk, tv, *to, prm, stream);
-    if (d == 64) return launch_d<64, false, kOutBoth>(tq, tk, tv, *to, prm, stream);
+    if (d == 128) return launch_d<128, kQkBf16, kOutBoth>(tq, tk, tv, *to, prm, stream);
+    if (d == 64) return launch_d<64, kQkBf16, kOutBoth>(tq, tk, tv, *to, prm, stream);
     return cudaErrorInvalidValue;
   }
   // statistics only: the output map is never used, tv stands in for it
-  if (d == 128) return launch_d<128, false, kOutStats>(tq, tk, tv, tv, prm, stream);
-  if (d == 64) return launch_d<64, false, kOutStats>(tq, tk, tv, tv, prm, stream);
+  if (d == 128) return launch_d<128, kQkBf16, kOutStats>(tq, tk, tv, tv, prm, stream);
+  if (d == 64) return launch_d<64, kQkBf16, kOutStats>(tq, tk, tv, tv, prm, stream);
   return cudaErrorInvalidValue;
 }
 

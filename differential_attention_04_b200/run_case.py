@@ -3,6 +3,7 @@
   python -m differential_attention_04_b200.run_case prefill --B 2 --N 4096 --H 12 --d 128 --causal 1 --iters 3
   python -m differential_attention_04_b200.run_case prefill --qk8 1 ...   (e4m3 queries/keys: quantise + forward;
                                                                           2: forward only; 3: quantise only)
+  python -m differential_attention_04_b200.run_case prefill --qk8 1 --bits 4 ...   (the same with e2m1 codes)
   python -m differential_attention_04_b200.run_case bwd --tc 1 ...   (tensor-core backward; 0: CUDA cores)
   python -m differential_attention_04_b200.run_case proj --B 1 --N 4096 --H 12 --d 128 --dmodel 3072 --iters 3
                                                                           (QKV projection + RoPE, then output projection)
@@ -32,6 +33,7 @@ def main(argv=None):
     ap.add_argument("--causal", type=int, default=1)
     ap.add_argument("--dtype", default="bf16")
     ap.add_argument("--qk8", type=int, default=0)
+    ap.add_argument("--bits", type=int, default=8, choices=[8, 4])
     ap.add_argument("--tc", type=int, default=1)
     ap.add_argument("--dmodel", type=int, default=3072)
     ap.add_argument("--S", type=int, default=64)
@@ -48,16 +50,17 @@ def main(argv=None):
         lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
         y = torch.empty_like(inp.v)
         if a.qk8:
-            qc, qs = api.quantize_qk(inp.q)
-            kc, ks = api.quantize_qk(inp.k)
+            quantize = api.quantize_qk if a.bits == 8 else api.quantize_qk4
+            forward = api.diffattn_fwd_qk8 if a.bits == 8 else api.diffattn_fwd_qk4
+            qc, qs = quantize(inp.q)
+            kc, ks = quantize(inp.k)
 
             def run():  # --qk8 1: quantise and forward; 2: forward only; 3: quantise only
                 if a.qk8 != 2:
-                    api.quantize_qk(inp.q, qc, qs)
-                    api.quantize_qk(inp.k, kc, ks)
+                    quantize(inp.q, qc, qs)
+                    quantize(inp.k, kc, ks)
                 if a.qk8 != 3:
-                    api.diffattn_fwd_qk8(qc, qs, kc, ks, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps,
-                                         inp.causal, out=y)
+                    forward(qc, qs, kc, ks, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
         else:
             run = lambda: api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps,
                                            inp.causal, out=y)

@@ -298,6 +298,42 @@ int diffattn_fwd_qk8(const void* q_codes, const float* q_scales,
                      float eps, int mode, cudaStream_t stream);
 
 /*
+ * diffattn_quantize_qk4 -- 4-bit codes (the peer review's 4-bit
+ * attention-logit quantisation, Fig. 8 of the paper): e2m1 codes of a bf16
+ * query or key tensor, with one absmax scale per (batch, head, map):
+ *
+ *   scales[b][h][i] = max |x[b, :, h, i, :]| / 6   (float32; 1 if that max is 0)
+ *   code(b, n, h, i, c) = e2m1(x[b, n, h, i, c] / scales[b][h][i])
+ *
+ * where e2m1 is the OCP Microscaling FP4 E2M1 encoding (bit 3 sign, 2
+ * exponent bits with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6), round to nearest even, saturating at +-6.  Two codes per byte:
+ * codes[b, n, h, i, j] = code(.., 2j) | code(.., 2j + 1) << 4.
+ * x      : bf16 [B, N, H, 2, d]
+ * codes  : device uint8 [B, N, H, 2, d / 2], written
+ * scales : device float32 [B][H][2], written (also used as scratch)
+ * d must be a multiple of 8; B * H * 2 <= 65535.  Three stream-ordered
+ * kernels and one memset; no allocation.
+ * Errors: DIFFATTN_ERR_INVALID_ARG, DIFFATTN_ERR_UNSUPPORTED, DIFFATTN_ERR_CUDA.
+ */
+int diffattn_quantize_qk4(const void* x, int B, int N, int H, int d, void* codes,
+                          float* scales, cudaStream_t stream);
+
+/*
+ * diffattn_fwd_qk4 -- diffattn_fwd_qk8 with e2m1 query and key codes (as
+ * diffattn_quantize_qk4 writes them, two per byte): the scores are a
+ * tensor-core product of the 4-bit codes (fp32 accumulation, exact) times
+ * q_scale * k_scale / sqrt(d).  q_codes and k_codes must be 32-byte aligned
+ * (DIFFATTN_ERR_INVALID_ARG otherwise); d must be 128.  Other arguments and
+ * errors as in diffattn_fwd_qk8.
+ */
+int diffattn_fwd_qk4(const void* q_codes, const float* q_scales,
+                     const void* k_codes, const float* k_scales,
+                     const void* v, void* o, int B, int N, int H, int d, int causal,
+                     const float* lambda, float lambda_init, const float* rms_w,
+                     float eps, int mode, cudaStream_t stream);
+
+/*
  * diffattn_decode_workspace_size -- bytes of device workspace that
  * diffattn_decode needs for S sequences of at most max_seqlen cached keys.
  * Returns 0 for invalid sizes.

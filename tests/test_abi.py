@@ -83,6 +83,17 @@ def test_validation_without_gpu(L):
     assert f8(fake, 16, 128, mode=5) == api.ERR_INVALID_ARG
     assert f8(nul, 16, 128) == api.ERR_INVALID_ARG
     assert f8(nul, 0, 128) == api.OK
+    # e2m1 queries/keys: same checks, and the codes must be 32-byte aligned
+    qz4 = lambda x, N, d, B=1, H=2: L.diffattn_quantize_qk4(x, B, N, H, d, x, x, nul)
+    assert qz4(fake, 16, 12) == api.ERR_INVALID_ARG
+    assert qz4(nul, 16, 128) == api.ERR_INVALID_ARG
+    assert qz4(fake, 16, 128, B=1 << 15, H=2) == api.ERR_UNSUPPORTED
+    f4 = lambda x, c, N, d, mode=0: L.diffattn_fwd_qk4(c, x, c, x, x, x, 1, N, 2, d, 1, x, 0.5, x, 1e-5, mode, nul)
+    assert f4(fake, fake, 16, 64) == api.ERR_UNSUPPORTED
+    assert f4(fake, fake, 16, 128, mode=5) == api.ERR_INVALID_ARG
+    assert f4(fake, ctypes.c_void_p(4096 + 16), 16, 128) == api.ERR_INVALID_ARG  # 16- but not 32-byte aligned
+    assert f4(nul, nul, 16, 128) == api.ERR_INVALID_ARG
+    assert f4(nul, nul, 0, 128) == api.OK
     # backward
     bw = lambda x, N, d, ws, wsb, mode=0: L.diffattn_bwd(x, x, x, x, api.F32, 1, N, 2, d, 1, x, 0.5, x, 1e-5, mode,
                                                          x, x, x, x, x, ws, wsb, nul)

@@ -14,10 +14,15 @@
 // x is [B, N, H, 2, d]; group g = (b * H + h) * 2 + i owns the d contiguous
 // elements of (b, n, h, i) for every n.  e4m3 codes take one byte each (rows
 // of d bytes); e2m1 codes two per byte, channel 2j in the low nibble (rows of
-// d / 2 bytes).  Each CTA takes one group and up to kTokPerCta tokens; every
-// row is d / 8 loads of 16 bytes.  HBM-bound: reads x twice (the second time
-// mostly from L2) and writes one byte (e4m3) or half a byte (e2m1) per
-// element.
+// d / 2 bytes).  HBM-bound: reads x twice (the second time mostly from L2)
+// and writes one byte (e4m3) or half a byte (e2m1) per element.
+//
+// Each CTA takes one group and up to kTokPerCta tokens; the grid runs the
+// token chunks of a group next to each other, so the CTAs resident at once
+// read whole token rows of neighbouring groups.  A row is d / 8 vectors of 16
+// bytes.  Every thread keeps one vector column and walks the rows with a
+// fixed stride (kThreadsQ / (d / 8) rows per pass), so the loop carries no
+// integer division; the e2m1 pass converts its values in pairs.
 #include <cuda_bf16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
@@ -48,6 +53,23 @@ __device__ __forceinline__ const uint4* row_ptr(const __nv_bfloat16* x, int b, i
   return reinterpret_cast<const uint4*>(x + ((static_cast<size_t>(b) * N + n) * (2 * H) + hi) * d);
 }
 
+// Thread layout over a chunk of `rows` rows of `vec` vectors: this thread's
+// first row and column, the row stride, and whether it takes part (all of
+// kThreadsQ do when vec divides it; for vec > kThreadsQ each thread walks
+// several columns of every row).
+struct Walk {
+  int r0, c0, r_step, c_step;
+  bool active;
+};
+__device__ __forceinline__ Walk walk_of(int vec) {
+  if (vec <= kThreadsQ) {
+    const int rpp = kThreadsQ / vec;
+    return {static_cast<int>(threadIdx.x) / vec, static_cast<int>(threadIdx.x) % vec, rpp, vec,
+            static_cast<int>(threadIdx.x) < rpp * vec};
+  }
+  return {0, static_cast<int>(threadIdx.x), 1, kThreadsQ, true};
+}
+
 __global__ void __launch_bounds__(kThreadsQ) qk_absmax_kernel(const __nv_bfloat16* __restrict__ x, int N, int H,
                                                               int d, unsigned int* __restrict__ amax_bits) {
   const int g = blockIdx.y;
@@ -55,21 +77,27 @@ __global__ void __launch_bounds__(kThreadsQ) qk_absmax_kernel(const __nv_bfloat1
   const int n0 = blockIdx.x * kTokPerCta;
   const int rows = min(N - n0, kTokPerCta);
   const int vec = d / 8;
-  const int total = rows * vec;
+  const Walk w = walk_of(vec);
+  const size_t row_vecs = static_cast<size_t>(2 * H) * vec;  // vectors from one token row to the next
   float m = 0.f;
-  for (int base = threadIdx.x; base < total; base += kUnroll * kThreadsQ) {
-    uint4 u[kUnroll];
+  if (w.active) {
+    for (int c = w.c0; c < vec; c += w.c_step) {
+      const uint4* p = row_ptr(x, b, n0, hi, N, H, d) + c;
+      for (int r = w.r0; r < rows; r += kUnroll * w.r_step) {
+        uint4 v[kUnroll];
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      const int idx = base + k * kThreadsQ;
-      u[k] = idx < total ? __ldg(row_ptr(x, b, n0 + idx / vec, hi, N, H, d) + idx % vec) : make_uint4(0, 0, 0, 0);
-    }
+        for (int k = 0; k < kUnroll; ++k) {
+          const int rr = r + k * w.r_step;
+          v[k] = rr < rows ? __ldg(p + rr * row_vecs) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      float f[8];
-      bf16x8_to_float(u[k], f);
+        for (int k = 0; k < kUnroll; ++k) {
+          float f[8];
+          bf16x8_to_float(v[k], f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+          for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+        }
+      }
     }
   }
 #pragma unroll
@@ -79,7 +107,7 @@ __global__ void __launch_bounds__(kThreadsQ) qk_absmax_kernel(const __nv_bfloat1
   __syncthreads();
   if (threadIdx.x == 0) {
     float t = wmax[0];
-    for (int w = 1; w < kThreadsQ / 32; ++w) t = fmaxf(t, wmax[w]);
+    for (int i = 1; i < kThreadsQ / 32; ++i) t = fmaxf(t, wmax[i]);
     atomicMax(amax_bits + g, __float_as_uint(t));
   }
 }
@@ -107,12 +135,15 @@ __device__ __forceinline__ uint2 encode8_e4m3(const float (&r)[8]) {
 }
 
 // 8 consecutive elements -> 8 e2m1 codes in 4 bytes, element j in nibble j
-// (the conversion saturates at +-6 and rounds to nearest even)
+// (the conversion saturates at +-6 and rounds to nearest even; a pair's
+// first element lands in the low nibble of its byte)
 __device__ __forceinline__ uint32_t encode8_e2m1(const float (&r)[8]) {
   uint32_t w = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    w |= (static_cast<uint32_t>(__nv_cvt_float_to_fp4(r[j], __NV_E2M1, cudaRoundNearest)) & 0xFu) << (4 * j);
+  for (int j = 0; j < 4; ++j)
+    w |= static_cast<uint32_t>(__nv_cvt_float2_to_fp4x2(make_float2(r[2 * j], r[2 * j + 1]), __NV_E2M1,
+                                                        cudaRoundNearest))
+         << (8 * j);
   return w;
 }
 
@@ -125,29 +156,35 @@ __global__ void __launch_bounds__(kThreadsQ) qk_quant_kernel(const __nv_bfloat16
   const int n0 = blockIdx.x * kTokPerCta;
   const int rows = min(N - n0, kTokPerCta);
   const int vec = d / 8;
+  const Walk w = walk_of(vec);
+  if (!w.active) return;
   const float s = __ldg(scales + g);
-  const int total = rows * vec;
-  for (int base = threadIdx.x; base < total; base += kUnroll * kThreadsQ) {
-    uint4 u[kUnroll];
+  const size_t row_vecs = static_cast<size_t>(2 * H) * vec;
+  constexpr int kOutBytes = BITS == 8 ? 8 : 4;  // code bytes per vector
+  for (int c = w.c0; c < vec; c += w.c_step) {
+    const uint4* p = row_ptr(x, b, n0, hi, N, H, d) + c;
+    uint8_t* q = codes + ((static_cast<size_t>(b) * N + n0) * (2 * H) + hi) * (vec * kOutBytes) + c * kOutBytes;
+    for (int r = w.r0; r < rows; r += kUnroll * w.r_step) {
+      uint4 v[kUnroll];
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      const int idx = base + k * kThreadsQ;
-      u[k] = idx < total ? __ldg(row_ptr(x, b, n0 + idx / vec, hi, N, H, d) + idx % vec) : make_uint4(0, 0, 0, 0);
-    }
+      for (int k = 0; k < kUnroll; ++k) {
+        const int rr = r + k * w.r_step;
+        v[k] = rr < rows ? __ldg(p + rr * row_vecs) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      const int idx = base + k * kThreadsQ;
-      if (idx >= total) break;
-      const int n = n0 + idx / vec, c = idx % vec;
-      float f[8];
-      bf16x8_to_float(u[k], f);
+      for (int k = 0; k < kUnroll; ++k) {
+        const int rr = r + k * w.r_step;
+        if (rr >= rows) break;
+        float f[8];
+        bf16x8_to_float(v[k], f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] = f[i] / s;
-      const size_t row = (static_cast<size_t>(b) * N + n) * (2 * H) + hi;
-      if constexpr (BITS == 8)
-        *reinterpret_cast<uint2*>(codes + row * d + 8 * c) = encode8_e4m3(f);
-      else
-        *reinterpret_cast<uint32_t*>(codes + row * (d / 2) + 4 * c) = encode8_e2m1(f);
+        for (int i = 0; i < 8; ++i) f[i] = f[i] / s;
+        uint8_t* dst = q + rr * row_vecs * kOutBytes;
+        if constexpr (BITS == 8)
+          *reinterpret_cast<uint2*>(dst) = encode8_e4m3(f);
+        else
+          *reinterpret_cast<uint32_t*>(dst) = encode8_e2m1(f);
+      }
     }
   }
 }

@@ -179,3 +179,15 @@ def test_workspace_size(L):
 def test_wait_limit_setter(L):
     assert L.diffattn_set_wait_limit_ns(-1) == api.ERR_INVALID_ARG
     assert L.diffattn_set_wait_limit_ns(0) == api.OK
+
+
+def test_package_exports_every_binding():
+    import inspect
+
+    import differential_attention_04_b200 as pkg
+
+    public = {n for n, f in inspect.getmembers(api, inspect.isfunction)
+              if f.__module__ == api.__name__ and not n.startswith("_")}
+    assert public, "no binding functions found"
+    missing = sorted(n for n in public if not hasattr(pkg, n))
+    assert not missing, f"not exported from the package: {missing}"

@@ -195,7 +195,7 @@ using namespace diffattn;
 
 extern "C" {
 
-int diffattn_version(void) { return 100; }
+int diffattn_version(void) { return 101; }  // 1.01: adds diffattn_quantize_qk4 and diffattn_fwd_qk4
 
 const char* diffattn_status_string(int s) {
   switch (s) {

@@ -440,7 +440,8 @@ int diffattn_set_wait_limit_ns(long long limit_ns);
 /* Human-readable name of a diffattn_status code. */
 const char* diffattn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor); 101 adds the 4-bit pair
+ * diffattn_quantize_qk4 / diffattn_fwd_qk4 to 100. */
 int diffattn_version(void);
 
 #ifdef __cplusplus

@@ -371,6 +371,44 @@ def _mut_decode_maps(q1, q2, k1, k2, v, lam, mode="diff"):
 
 _orig_head = ref.diffattn_head_prenorm
 _orig_decode = ref.decode_head_prenorm
+_orig_fwd = ref.diffattn_fwd
+_orig_norm = ref.headwise_rmsnorm
+
+
+def _mut_norm_over_tokens(O, w, eps, lambda_init):
+    O = np.asarray(O, dtype=np.float64)
+    ms = np.mean(O * O, axis=0, keepdims=True)  # over the rows instead of the head's channels
+    return (1.0 - float(lambda_init)) * np.asarray(w, dtype=np.float64) * O / np.sqrt(ms + float(eps))
+
+
+def _mut_weight_reversed(O, w, eps, lambda_init):
+    return _orig_norm(O, np.asarray(w)[::-1], eps, lambda_init)
+
+
+def _mut_v_next_head(q, k, v, lam, lambda_init, w, eps, causal, rows=None, heads=None, mode="diff"):
+    return _orig_fwd(q, k, np.roll(np.asarray(v), -1, axis=2), lam, lambda_init, w, eps, causal, rows, heads, mode)
+
+
+def _mut_query_maps_swapped(q, k, v, lam, lambda_init, w, eps, causal, rows=None, heads=None, mode="diff"):
+    return _orig_fwd(np.asarray(q)[:, :, :, ::-1, :], k, v, lam, lambda_init, w, eps, causal, rows, heads, mode)
+
+
+def _mut_rows_lose_positions(q1, k1, q2, k2, v, lam, causal, rows=None, mode="diff"):
+    if rows is None:
+        return _orig_head(q1, k1, q2, k2, v, lam, causal, rows, mode)
+    q1, q2 = np.asarray(q1, np.float64), np.asarray(q2, np.float64)
+    rows = np.asarray(rows)
+    scale = 1.0 / math.sqrt(q1.shape[1])
+    pos = np.arange(len(rows))  # the sampled rows masked as if they were rows 0, 1, ...
+    S1 = ref._causal_scores(q1[rows], np.asarray(k1, np.float64), scale, pos, causal)
+    S2 = ref._causal_scores(q2[rows], np.asarray(k2, np.float64), scale, pos, causal)
+    return ref.map_weights(S1, S2, lam, mode) @ np.asarray(v, np.float64)
+
+
+def _mut_scale_value_width(q1, k1, q2, k2, v, lam, causal, rows=None, mode="diff"):
+    f = math.sqrt(0.5)  # 1/sqrt(2d): the value width instead of the per-map width
+    return _orig_head(np.asarray(q1, np.float64) * f, k1, np.asarray(q2, np.float64) * f, k2, v, lam, causal, rows,
+                      mode)
 
 MUTANTS = {
     "plus_lambda": ("diff_weights", _mut_sign),
@@ -387,6 +425,12 @@ MUTANTS = {
     "decode_map2_uses_k1": ("decode_head_prenorm", _mut_decode_maps),
     "sum_mode_subtracts": ("map_weights", _mut_sum_subtracts),
     "lambda_zero_keeps_map2": ("map_weights", _mut_zero_keeps_map2),
+    "norm_over_tokens": ("headwise_rmsnorm", _mut_norm_over_tokens),
+    "norm_weight_reversed": ("headwise_rmsnorm", _mut_weight_reversed),
+    "values_of_next_head": ("diffattn_fwd", _mut_v_next_head),
+    "query_maps_swapped": ("diffattn_fwd", _mut_query_maps_swapped),
+    "sampled_rows_lose_positions": ("diffattn_head_prenorm", _mut_rows_lose_positions),
+    "scale_1_over_sqrt_value_width": ("diffattn_head_prenorm", _mut_scale_value_width),
 }
 
 

@@ -188,3 +188,21 @@ def test_pins_catch_mutant(name, monkeypatch):
         except (AssertionError, FloatingPointError, ValueError):
             caught.append(pin.__name__)
     assert caught, f"no pin catches mutant {name}"
+
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=30, deadline=None)
+@given(B=st.integers(1, 2), N=st.integers(1, 6), H=st.integers(1, 2), d=st.integers(1, 4), causal=st.booleans(),
+       mode=st.sampled_from(["diff", "lambda_zero", "sum"]), lam=st.floats(-1.5, 1.5),
+       lam_init=st.floats(0.0, 0.9), eps=st.sampled_from([1e-5, 0.1]), scale=st.sampled_from([0.3, 1.0, 3.0]),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_autograd_on_random_shapes(B, N, H, d, causal, mode, lam, lam_init, eps, scale, seed):
+    # pin_autograd over drawn shapes (one token and one channel included), masks, modes and lambda
+    q, k, v, dy, w = _case(seed, B=B, N=N, H=H, d=d, scale=scale)
+    got = bwd.diffattn_bwd(q, k, v, dy, lam, lam_init, w, eps, causal, mode)
+    want = _torch_grads(q, k, v, dy, lam, lam_init, w, eps, causal, mode)
+    for name, g, t in zip(("dq", "dk", "dv", "dlam", "dw"), got, want):
+        assert _close(g, t, tol=1e-8), name

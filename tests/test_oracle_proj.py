@@ -175,3 +175,36 @@ def test_pins_catch_mutant(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             caught.append(pin.__name__)
     assert caught, f"no pin catches mutant {name}"
+
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(B=st.integers(1, 2), N=st.integers(1, 5), H=st.integers(1, 2), half=st.integers(1, 3), dm=st.integers(1, 6),
+       base=st.sampled_from([100.0, 10000.0]), seed=st.integers(0, 2 ** 31 - 1))
+def test_projection_with_rope_matches_loops(B, N, H, half, dm, base, seed):
+    # the fused projection + rotation over drawn shapes, against loops that rotate each
+    # consecutive channel pair of Q1, Q2, K1, K2 by n * base^(-2j/d), n the token's position
+    d = 2 * half
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B * N, dm))
+    w = rng.standard_normal((3 * H * 2 * d, dm))
+    q, k, v = pr.qkv_proj(x, w, B, N, H, d, rope_base=base)
+    for b in range(B):
+        for n in range(N):
+            row = b * N + n
+            feat = [sum(x[row, t] * w[f, t] for t in range(dm)) for f in range(w.shape[0])]
+            for h in range(H):
+                for i in range(2):
+                    for part, got in ((0, q), (1, k)):
+                        f0 = part * H * 2 * d + (h * 2 + i) * d
+                        for j in range(half):
+                            a, c = feat[f0 + 2 * j], feat[f0 + 2 * j + 1]
+                            ang = n * base ** (-2.0 * j / d)
+                            want = (a * math.cos(ang) - c * math.sin(ang), a * math.sin(ang) + c * math.cos(ang))
+                            assert abs(got[b, n, h, i, 2 * j] - want[0]) < 1e-9
+                            assert abs(got[b, n, h, i, 2 * j + 1] - want[1]) < 1e-9
+                for c2 in range(2 * d):
+                    assert abs(v[b, n, h, c2] - feat[2 * H * 2 * d + h * 2 * d + c2]) < 1e-9

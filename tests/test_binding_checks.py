@@ -52,8 +52,17 @@ def test_valid_patterns_reach_the_device_check(pre):
     _cpu_only(api.diffattn_fwd_qk8, codes8, sc, codes8, sc, pre.v, lam, 0.5, pre.rms_w, 1e-5, True,
               out=torch.empty_like(pre.v))
     _cpu_only(api.diffattn_fwd_qk4, codes4, sc, codes4, sc, pre.v, lam, 0.5, pre.rms_w, 1e-5, True)
+    _cpu_only(api.quantize_qk, pre.q, codes8, sc)  # into the caller's buffers, as the bench loop does
+    _cpu_only(api.quantize_qk4, pre.q, codes4, sc)
+    _cpu_only(api.diffattn_fwd_qk4, codes4, sc, codes4, sc, pre.v, lam, 0.5, pre.rms_w, 1e-5, True,
+              out=torch.empty_like(pre.v))
     dy = torch.zeros_like(pre.v)
     _cpu_only(api.diffattn_bwd, pre.q, pre.k, pre.v, dy, lam, 0.5, pre.rms_w)
+    _cpu_only(api.diffattn_bwd, pre.q, pre.k, pre.v, dy, lam, 0.5, pre.rms_w, 1e-5, True,
+              workspace=torch.empty(64, dtype=torch.uint8))
+    f32in = wl.make_prefill(1, 12, 2, 48, causal=False, dtype="f32", seed=3, device="cpu")
+    _cpu_only(api.diffattn_fwd, f32in.q, f32in.k, f32in.v, lam, 0.5, f32in.rms_w, 1e-5, False)
+    _cpu_only(api.diffattn_bwd, f32in.q, f32in.k, f32in.v, torch.zeros_like(f32in.v), lam, 0.5, f32in.rms_w)
     outs = (torch.empty(pre.q.shape, **f32), torch.empty(pre.k.shape, **f32), torch.empty(pre.v.shape, **f32),
             torch.empty(1, **f32), torch.empty(2 * d, **f32))
     ws = torch.empty(64, dtype=torch.uint8)

@@ -37,6 +37,10 @@ METRIC = "DiffAttn fwd TFLOP/s & % BF16 tensor peak (prefill); decode HBM GB/s, 
 WORKLOAD = "prefill_3b"
 DECODE_WORKLOAD = "decode_64x12"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures (dense bf16 tensor rate, HBM3e bandwidth), reported beside the measured ones
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+# the other prefill configurations timed beside the headline one: (workload, timed steps)
+PREFILL_SUBCASES = (("prefill_64k_needle", 10), ("prefill_13b_causal", 150), ("prefill_13b_nomask", 100))
 
 
 def parse_args(argv=None):
@@ -56,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-proj", action="store_true")
     ap.add_argument("--proj-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other prefill configurations")
+    ap.add_argument("--no-small", action="store_true", help="skip the latency-bound small prefill")
     ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     return ap.parse_args(argv)
@@ -102,21 +108,30 @@ def prefill_row_flops(N, d, causal, convention):
 
 
 def read_profile_traffic(kernel_tag: str):
-    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current kernel source."""
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current kernel source.
+
+    The summary names the sources it was captured on (`source_files:`, paths
+    under csrc/, comma-separated; the prefill or decode kernel's file when
+    absent) and their hash (`source_sha256_16`: sha256 of the files' bytes in
+    that order); a summary of older sources gives None."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
-    src = os.path.join(ROOT, "differential_attention_04_b200", "csrc",
-                       "prefill_sm100.cu" if kernel_tag.startswith("prefill") else "decode.cu")
-    if not (os.path.exists(path) and os.path.exists(src)):
+    if not os.path.exists(path):
         return None
-    want = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     vals = {}
     for line in open(path):
-        if ":" in line:
+        if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("source_sha256_16") != want:
+    names = vals.get("source_files") or ("prefill_sm100.cu" if kernel_tag.startswith("prefill") else "decode.cu")
+    h = hashlib.sha256()
+    for name in (x.strip() for x in names.split(",")):
+        src = os.path.join(ROOT, "differential_attention_04_b200", "csrc", name)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    if vals.get("source_sha256_16") != h.hexdigest()[:16]:
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])
@@ -131,8 +146,9 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,timestamp")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         self.gpu = gpu_index
+        self.period_ms = period_ms
         self.proc = None
         self.path = None
         self.t_begin = self.t_end = None
@@ -151,7 +167,7 @@ class ClockSampler:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+                 "-lms", str(self.period_ms)], stdout=self.out, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -181,8 +197,15 @@ class ClockSampler:
                 except ValueError:
                     return None
             inside = [r for r in rows if stamp(r) is not None and self.t_begin <= stamp(r) <= self.t_end]
+            within = bool(inside)
             if inside:
                 rows = inside
+            else:  # a region shorter than the sampling period: keep the samples around it
+                near = [r for r in rows if stamp(r) is not None and
+                        self.t_begin - 0.25 <= stamp(r) <= self.t_end + 0.25]
+                rows = near or rows
+        else:
+            within = False
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -195,7 +218,27 @@ class ClockSampler:
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(pw) if pw else None,
                 "power_w_median": statistics.median(pw) if pw else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "inside_timed_region": within,
+                "period_ms": self.period_ms}
+
+
+def sampled(gpu_index: int, loop):
+    """Run `loop()` (a timed loop that synchronises before it returns) with the
+    SM clocks sampled around it; returns (loop's result, clocks, wall seconds)."""
+    clk = ClockSampler(gpu_index)
+    clk.start()
+    clk.mark_begin()
+    t = time.perf_counter()
+    r = loop()
+    wall = time.perf_counter() - t
+    clk.mark_end()
+    return r, clk.stop(), wall
+
+
+def spec_fracs(achieved: float, unit: str) -> dict:
+    """Fraction of the nominal B200 figure for the same quantity."""
+    spec = SPEC_PEAKS["bf16_tflops"] if unit == "TFLOP/s" else SPEC_PEAKS["hbm_gbs"]
+    return {"frac_of_spec": achieved / spec, "spec_peak": spec}
 
 
 def blas_threads():
@@ -241,7 +284,8 @@ def cpu_baseline(inp, budget_s):
         secs += t
         seed += 1
     flops = rows_total * prefill_row_flops(N, d, inp.causal, "metric")
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "host_cpu_count": os.cpu_count(), "kind": "oracle",
             "sample": f"{rows_total} query rows (each against all {N} keys, both maps materialised) of "
                       f"{seed} seeded (batch, head) pairs of the {WORKLOAD} workload, {secs:.1f} s of CPU work; "
                       f"FLOPs per row counted with the metric convention 16*N*d/2"}
@@ -275,11 +319,15 @@ def bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, K):
     torch.cuda.synchronize()
     barrier()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for a, b in ev:
-        a.record()
-        step()
-        b.record()
-    torch.cuda.synchronize()
+
+    def loop():
+        for a, b in ev:
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+
+    _, clk, wall = sampled(inp.q.device.index, loop)
     ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev))
     pairs = B * H * (N * (N + 1) // 2 if inp.causal else N * N)
     # algorithmic: per visible (query, key) pair, 20 d flops -- both maps' scores
@@ -326,12 +374,14 @@ def bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, K):
                               "note": "diffattn_fwd_train (output + each map's A_i V and log-sum-exp) then "
                                       "diffattn_bwd_tc_saved (no statistics pass)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": read_profile_traffic("bwd_grad_sm100_bwd_3b"),
+                         **spec_fracs(achieved, "TFLOP/s"),
                          "executed_tflops": executed / (ms * 1e-3) / 1e12,
                          "kernel": "prefill_sm100_kernel (statistics mode) + bwd_prep + bwd_grad_sm100 x3 (dV, dK, dQ)",
                          "peak_source": f"{peak_src} bf16 dense, " + (
                              f"sustained (timed loop {loop_ms / 1e3:.2f} s)" if sustained
                              else f"burst (timed loop {loop_ms / 1e3:.2f} s)")},
+            "clocks": clk, "loop_wall_s": wall,
             "gpu_launches": 10 * K}
 
 
@@ -359,13 +409,17 @@ def bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, K):
     torch.cuda.synchronize()
     barrier()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    for e0, e1, e2 in ev:
-        e0.record()
-        api.qkv_proj(inp.x, inp.w_qkv, B, N, H, d, table, out=qkv)
-        e1.record()
-        api.out_proj(qkv[2], inp.w_o, out=y)
-        e2.record()
-    torch.cuda.synchronize()
+
+    def loop():
+        for e0, e1, e2 in ev:
+            e0.record()
+            api.qkv_proj(inp.x, inp.w_qkv, B, N, H, d, table, out=qkv)
+            e1.record()
+            api.out_proj(qkv[2], inp.w_o, out=y)
+            e2.record()
+        torch.cuda.synchronize()
+
+    _, clk, wall = sampled(dev.index, loop)
     q_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b, _ in ev))
     o_ms = reduce_max(statistics.mean(b.elapsed_time(c) for _, b, c in ev))
     M = B * N
@@ -379,10 +433,12 @@ def bench_proj(api, wl, dev, peaks, peak_src, reduce_max, barrier, K):
             "unit": "TFLOP/s", "steps": K, "ms_per_step": q_ms + o_ms, "qkv_rope_ms": q_ms, "out_proj_ms": o_ms,
             "qkv_tflops": f_qkv / (q_ms * 1e-3) / 1e12, "out_tflops": f_o / (o_ms * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "proj_gemm_sm100_kernel (x2)",
+                         "frac": achieved / peak, "traffic": read_profile_traffic("proj_gemm_sm100_proj_3b"),
+                         **spec_fracs(achieved, "TFLOP/s"), "kernel": "proj_gemm_sm100_kernel (x2)",
                          "peak_source": f"{peak_src} bf16 dense, " + (
                              f"sustained (timed loop {loop_ms / 1e3:.2f} s)" if sustained
                              else f"burst (timed loop {loop_ms / 1e3:.2f} s)")},
+            "clocks": clk, "loop_wall_s": wall,
             "gpu_launches": 2 * K}
 
 
@@ -413,13 +469,17 @@ def bench_lowbit(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K, bits
     torch.cuda.synchronize()
     barrier()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    for e0, e1, e2 in ev:
-        e0.record()
-        quant()
-        e1.record()
-        fwd()
-        e2.record()
-    torch.cuda.synchronize()
+
+    def loop():
+        for e0, e1, e2 in ev:
+            e0.record()
+            quant()
+            e1.record()
+            fwd()
+            e2.record()
+        torch.cuda.synchronize()
+
+    _, clk, wall = sampled(inp.q.device.index, loop)
     q_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b, _ in ev))
     f_ms = reduce_max(statistics.mean(b.elapsed_time(c) for _, b, c in ev))
     flops_metric = prefill_flops(B, N, H, d, inp.causal, "metric")
@@ -434,10 +494,123 @@ def bench_lowbit(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, K, bits
             "value": flops_metric / ((q_ms + f_ms) * 1e-3) / 1e12, "unit": "TFLOP/s", "steps": K,
             "ms_per_step": q_ms + f_ms, "quantize_ms": q_ms, "prefill_ms": f_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": mixed, "unit": "TFLOP/s",
-                         "frac": achieved / mixed, "traffic": None, "kernel": f"prefill_sm100_kernel<128, {fmt}>",
+                         "frac": achieved / mixed, "traffic": read_profile_traffic(f"prefill_sm100_{fmt}_prefill_3b"),
+                         "frac_of_spec": achieved / (1.2 * SPEC_PEAKS["bf16_tflops"]),
+                         "spec_peak": 1.2 * SPEC_PEAKS["bf16_tflops"],
+                         "kernel": f"prefill_sm100_kernel<128, {fmt}>",
                          "peak_source": f"{peak_src} bf16 dense (burst) x 1.2: scores on the f8f6f4 path at the "
                                         "nominal 2x rate"},
+            "clocks": clk, "loop_wall_s": wall,
             "gpu_launches": 7 * K}
+
+
+def bench_prefill_case(api, wl, dev, name, K, peaks, peak_src, reduce_max, barrier, rank):
+    """Another prefill configuration: lambda + prefill, K timed steps with CUDA
+    events around each prefill launch and the SM clocks sampled during the loop."""
+    import torch
+
+    inp = wl.make_prefill_case(name, seed=rank_seed(1234, rank), device=dev)
+    B, N, H, _, d = inp.q.shape
+    lam = torch.empty(1, dtype=torch.float32, device=dev)
+    y = torch.empty_like(inp.v)
+
+    def step(e=None):
+        api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init, out=lam)
+        if e is not None:
+            e[0].record()
+        api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal, out=y)
+        if e is not None:
+            e[1].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def loop():
+        t0.record()
+        for e in ev:
+            step(e)
+        t1.record()
+        torch.cuda.synchronize()
+
+    _, clk, wall = sampled(dev.index, loop)
+    status = api.device_status()
+    if status != api.OK:
+        raise SystemExit(f"kernel status {status} in {name}")
+    kern_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev))
+    loop_ms = reduce_max(t0.elapsed_time(t1))
+    flops_metric = prefill_flops(B, N, H, d, inp.causal, "metric")
+    flops_alg = prefill_flops(B, N, H, d, inp.causal, "algorithmic")
+    achieved = flops_alg / (kern_ms * 1e-3) / 1e12
+    sustained = loop_ms >= 1000.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    out = {
+        "workload": f"{name}: B={B} N={N} H={H} d={d} V width {2 * d} {'causal' if inp.causal else 'no mask'} bf16",
+        "value": job_throughput(flops_metric, int(os.environ.get("WORLD_SIZE", "1")), loop_ms / K) / 1e12,
+        "unit": "TFLOP/s", "steps": K, "kernel_ms": kern_ms, "ms_per_step": loop_ms / K,
+        "flops_per_step_algorithmic": flops_alg, "flops_per_step_metric": flops_metric,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": read_profile_traffic(f"prefill_sm100_{name}"),
+                     "frac_of_burst": achieved / peaks["bf16_tflops"],
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                     **spec_fracs(achieved, "TFLOP/s"), "kernel": "prefill_sm100_kernel<128>",
+                     "peak_source": f"{peak_src} bf16 dense, " + (
+                         f"sustained (timed loop {loop_ms / 1e3:.2f} s)" if sustained
+                         else f"burst (timed loop {loop_ms / 1e3:.2f} s < 1 s)")},
+        "clocks": clk, "loop_wall_s": wall, "gpu_launches": 2 * K,
+    }
+    del inp, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_small_prefill(api, wl, dev, reduce_max, barrier, rank, K=400):
+    """A latency-bound prefill (B=1, H=12, N=512, causal, bf16): the host time
+    one diffattn_fwd call takes (argument checks, tensor-map set-up, launch),
+    measured as the wall time of K back-to-back calls that the GPU never holds
+    up, beside the device time per launch."""
+    import torch
+
+    inp = wl.make_prefill(1, 512, 12, 128, causal=True, dtype="bf16", lambda_init=0.5, seed=rank_seed(77, rank),
+                          device=dev)
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+    y = torch.empty_like(inp.v)
+    from differential_attention_04_b200._lib import lib
+
+    L = lib()
+    B, N, H, _, d = inp.q.shape
+    args = (inp.q.data_ptr(), inp.k.data_ptr(), inp.v.data_ptr(), y.data_ptr(), api.BF16, B, N, H, d, 1,
+            lam.data_ptr(), inp.lambda_init, inp.rms_w.data_ptr(), inp.eps, torch.cuda.current_stream().cuda_stream)
+    for _ in range(20):
+        assert L.diffattn_fwd(*args) == api.OK
+    torch.cuda.synchronize()
+    barrier()
+    # host cost per call through the C ABI (ctypes marshalling included), with
+    # the GPU queue kept short so that no call waits for the device
+    host_us = []
+    for _ in range(5):
+        t = time.perf_counter()
+        for _ in range(K // 5):
+            L.diffattn_fwd(*args)
+        host_us.append((time.perf_counter() - t) / (K // 5) * 1e6)
+        torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(K):
+        L.diffattn_fwd(*args)
+    b.record()
+    torch.cuda.synchronize()
+    dev_ms = reduce_max(a.elapsed_time(b)) / K
+    flops_alg = prefill_flops(B, N, H, d, True, "algorithmic")
+    return {"workload": f"B={B} N={N} H={H} d={d} causal bf16 (latency-bound)",
+            "host_us_per_call": statistics.median(host_us), "host_us_per_call_all": host_us,
+            "device_ms_per_launch": dev_ms, "achieved_tflops_algorithmic": flops_alg / (dev_ms * 1e-3) / 1e12,
+            "how": "host: wall time of back-to-back diffattn_fwd calls through ctypes, no synchronisation inside; "
+                   "device: CUDA events around K back-to-back launches",
+            "gpu_launches": K + 20 + K}
 
 
 def run_reference(args):
@@ -469,7 +642,8 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": prefill_config(inp, args.workload, args.gpus, prefill_flops(*inp.q.shape[:3], d, inp.causal, "metric"),
                                  prefill_flops(*inp.q.shape[:3], d, inp.causal, "algorithmic")),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "host_cpu_count": os.cpu_count(), "kind": "oracle",
                          "sample": f"{rows} query rows per step (each against all {N} keys) of one seeded "
                                    f"(batch, head) of {args.workload}"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -645,7 +819,8 @@ def run_ours(args):
                      "kernel": "prefill_sm100_kernel<128>", "kernel_ms": kern_ms,
                      "peak_source": f"{peak_src} bf16 dense, {peak_kind}",
                      "frac_of_burst": achieved / peaks["bf16_tflops"],
-                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                     **spec_fracs(achieved, "TFLOP/s")},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "steps": E,
                 "how": "pinned host inputs copied up and the output read back every step, through diffattn_lambda "
@@ -654,6 +829,13 @@ def run_ours(args):
         "clocks": clk,
     }
 
+    if not args.no_configs and args.workload == WORKLOAD:
+        line["configs"] = {}
+        for name, steps in PREFILL_SUBCASES:
+            line["configs"][name] = bench_prefill_case(api, wl, dev, name, steps, peaks, peak_src, reduce_max,
+                                                       barrier, rank)
+    if not args.no_small:
+        line["small_prefill"] = bench_small_prefill(api, wl, dev, reduce_max, barrier, rank)
     if not args.no_bwd:
         line["bwd"] = bench_bwd(api, inp, lam, peaks, peak_src, reduce_max, barrier, args.bwd_steps)
     if not args.no_proj:
@@ -695,11 +877,15 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world
     torch.cuda.synchronize()
     barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        step()
-    b.record()
-    torch.cuda.synchronize()
+
+    def loop():
+        a.record()
+        for _ in range(steps):
+            step()
+        b.record()
+        torch.cuda.synchronize()
+
+    _, clk, wall = sampled(dev.index, loop)
     ms = reduce_max(a.elapsed_time(b)) / steps
     kv_bytes = T * H * (2 * d + 2 * d) * 2
     io_bytes = S * H * 2 * d * 2 * 2
@@ -711,9 +897,10 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world
         "workload": f"{DECODE_WORKLOAD}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
                     f"({kv_bytes / 1e9:.2f} GB per step)",
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": traffic,
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, **spec_fracs(gbs, "GB/s"),
                      "kernel": "decode_partial_kernel + decode_combine_kernel",
                      "algorithmic_bytes": alg, "peak_source": f"{peak_src} HBM copy"},
+        "clocks": clk, "loop_wall_s": wall,
         "gpu_launches": 2 * steps,
     }
 

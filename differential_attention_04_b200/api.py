@@ -34,16 +34,29 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _stream() -> int:
-    return torch.cuda.current_stream().cuda_stream
-
-
-def _dev(*ts: torch.Tensor) -> None:
+def _dev(*ts: torch.Tensor) -> torch.device:
+    """The one CUDA device all of `ts` live on (every tensor contiguous)."""
+    dev = None
     for t in ts:
         if not t.is_cuda:
             raise ValueError("all tensors must be CUDA tensors")
         if not t.is_contiguous():
             raise ValueError("all tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"all tensors must be on one device (found {dev} and {t.device})")
+    return dev
+
+
+def _launch(name: str, tensors, *args) -> None:
+    """Call the C entry point `name` with `args` and the current stream of the
+    device that `tensors` (every tensor the call reads or writes) live on, with
+    that device current: the library launches on the current device."""
+    dev = _dev(*tensors)
+    with torch.cuda.device(dev):
+        status = getattr(lib(), name)(*args, torch.cuda.current_stream(dev).cuda_stream)
+    _check(name, status)
 
 
 # Shape and dtype checks run before the device check, so that every tensor the
@@ -83,9 +96,8 @@ def diffattn_lambda(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor, lk2
     if out is None:
         out = torch.empty(1, dtype=torch.float32, device=lq1.device)
     _scalar_f32("out", out)
-    _dev(lq1, lk1, lq2, lk2, out)
-    _check("diffattn_lambda", lib().diffattn_lambda(
-        _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), lq1.numel(), float(lambda_init), _ptr(out), _stream()))
+    _launch("diffattn_lambda", (lq1, lk1, lq2, lk2, out),
+            _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), lq1.numel(), float(lambda_init), _ptr(out))
     return out
 
 
@@ -110,15 +122,13 @@ def diffattn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.T
     if out is None:
         out = torch.empty_like(v)
     _like("out", out, v.shape, v.dtype)
-    _dev(q, k, v, lam, rms_w, out)
+    ts = (q, k, v, lam, rms_w, out)
     if mode == MODE_DIFF:
-        _check("diffattn_fwd", lib().diffattn_fwd(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)), _ptr(lam),
-            float(lambda_init), _ptr(rms_w), float(eps), _stream()))
+        _launch("diffattn_fwd", ts, _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)),
+                _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps))
     else:
-        _check("diffattn_fwd_mode", lib().diffattn_fwd_mode(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)), _ptr(lam),
-            float(lambda_init), _ptr(rms_w), float(eps), int(mode), _stream()))
+        _launch("diffattn_fwd_mode", ts, _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, B, N, H, d, int(bool(causal)),
+                _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode))
     return out
 
 
@@ -136,9 +146,8 @@ def quantize_qk(x: torch.Tensor, codes: torch.Tensor | None = None,
     if codes.shape != x.shape or codes.dtype != torch.uint8 or scales.numel() != B * H * 2 or \
             scales.dtype != torch.float32:
         raise ValueError("codes must be uint8 like x and scales float32 [B, H, 2]")
-    _dev(x, codes, scales)
-    _check("diffattn_quantize_qk", lib().diffattn_quantize_qk(_ptr(x), B, N, H, d, _ptr(codes), _ptr(scales),
-                                                              _stream()))
+    _launch("diffattn_quantize_qk", (x, codes, scales),
+            _ptr(x), B, N, H, d, _ptr(codes), _ptr(scales))
     return codes, scales
 
 
@@ -162,10 +171,9 @@ def diffattn_fwd_qk8(q_codes: torch.Tensor, q_scales: torch.Tensor, k_codes: tor
     if out is None:
         out = torch.empty_like(v)
     _like("out", out, v.shape, torch.bfloat16)
-    _dev(q_codes, q_scales, k_codes, k_scales, v, lam, rms_w, out)
-    _check("diffattn_fwd_qk8", lib().diffattn_fwd_qk8(
-        _ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v), _ptr(out), B, N, H, d,
-        int(bool(causal)), _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode), _stream()))
+    _launch("diffattn_fwd_qk8", (q_codes, q_scales, k_codes, k_scales, v, lam, rms_w, out),
+            _ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v), _ptr(out), B, N, H, d,
+            int(bool(causal)), _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode))
     return out
 
 
@@ -186,9 +194,8 @@ def quantize_qk4(x: torch.Tensor, codes: torch.Tensor | None = None,
     if tuple(codes.shape) != shape or codes.dtype != torch.uint8 or scales.numel() != B * H * 2 or \
             scales.dtype != torch.float32:
         raise ValueError("codes must be uint8 [B, N, H, 2, d / 2] and scales float32 [B, H, 2]")
-    _dev(x, codes, scales)
-    _check("diffattn_quantize_qk4", lib().diffattn_quantize_qk4(_ptr(x), B, N, H, d, _ptr(codes), _ptr(scales),
-                                                                _stream()))
+    _launch("diffattn_quantize_qk4", (x, codes, scales),
+            _ptr(x), B, N, H, d, _ptr(codes), _ptr(scales))
     return codes, scales
 
 
@@ -206,10 +213,9 @@ def diffattn_fwd_qk4(q_codes: torch.Tensor, q_scales: torch.Tensor, k_codes: tor
     if out is None:
         out = torch.empty_like(v)
     _like("out", out, v.shape, torch.bfloat16)
-    _dev(q_codes, q_scales, k_codes, k_scales, v, lam, rms_w, out)
-    _check("diffattn_fwd_qk4", lib().diffattn_fwd_qk4(
-        _ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v), _ptr(out), B, N, H, d,
-        int(bool(causal)), _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode), _stream()))
+    _launch("diffattn_fwd_qk4", (q_codes, q_scales, k_codes, k_scales, v, lam, rms_w, out),
+            _ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v), _ptr(out), B, N, H, d,
+            int(bool(causal)), _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode))
     return out
 
 
@@ -235,11 +241,10 @@ def diffattn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch.Te
     need = bwd_workspace_size(B, N, H, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    _dev(workspace)
-    _check("diffattn_bwd", lib().diffattn_bwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(dy), dt, B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
-        _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream()))
+    _launch("diffattn_bwd", (q, k, v, dy, lam, rms_w, dq, dk, dv, dlam, dw, workspace),
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dy), dt, B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+            _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
+            workspace.numel() * workspace.element_size())
     return dq, dk, dv, dlam, dw
 
 
@@ -278,11 +283,10 @@ def diffattn_bwd_tc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy: torch
     _dev(q, k, v, dy, lam, rms_w)
     if workspace is None:
         workspace = torch.empty(bwd_tc_workspace_size(B, N, H, d), dtype=torch.uint8, device=q.device)
-    _dev(workspace)
-    _check("diffattn_bwd_tc", lib().diffattn_bwd_tc(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(dy), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
-        _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream()))
+    _launch("diffattn_bwd_tc", (q, k, v, dy, lam, rms_w, dq, dk, dv, dlam, dw, workspace),
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dy), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+            _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
+            workspace.numel() * workspace.element_size())
     return dq, dk, dv, dlam, dw
 
 
@@ -301,10 +305,9 @@ def diffattn_fwd_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: t
     _like("out", out, v.shape, torch.bfloat16)
     if workspace is None:
         workspace = torch.empty(bwd_tc_workspace_size(B, N, H, d), dtype=torch.uint8, device=q.device)
-    _dev(q, k, v, lam, rms_w, out, workspace)
-    _check("diffattn_fwd_train", lib().diffattn_fwd_train(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
-        _ptr(rms_w), float(eps), int(mode), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()))
+    _launch("diffattn_fwd_train", (q, k, v, lam, rms_w, out, workspace),
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+            _ptr(rms_w), float(eps), int(mode), _ptr(workspace), workspace.numel() * workspace.element_size())
     return out, workspace
 
 
@@ -318,18 +321,17 @@ def diffattn_bwd_tc_saved(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dy:
     _scalar_f32("lam", lam)
     _f32("rms_w", rms_w, 2 * d)
     dq, dk, dv, dlam, dw = _grads_out(out, q, v, d)
-    _dev(q, k, v, dy, lam, rms_w, workspace)
-    _check("diffattn_bwd_tc_saved", lib().diffattn_bwd_tc_saved(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(dy), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
-        _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream()))
+    _launch("diffattn_bwd_tc_saved", (q, k, v, dy, lam, rms_w, dq, dk, dv, dlam, dw, workspace),
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dy), B, N, H, d, int(bool(causal)), _ptr(lam), float(lambda_init),
+            _ptr(rms_w), float(eps), int(mode), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(dw), _ptr(workspace),
+            workspace.numel() * workspace.element_size())
     return dq, dk, dv, dlam, dw
 
 
 def rope_table(N: int, d: int, base: float = 10000.0, device=None) -> torch.Tensor:
     """(cos, sin) of n * base^(-2j/d) for n < N, j < d/2: float32 [N, d/2, 2] on the device."""
     t = torch.empty((N, d // 2, 2), dtype=torch.float32, device=device or torch.device("cuda"))
-    _check("diffattn_rope_table", lib().diffattn_rope_table(int(N), int(d), float(base), _ptr(t), _stream()))
+    _launch("diffattn_rope_table", (t,), int(N), int(d), float(base), _ptr(t))
     return t
 
 
@@ -353,10 +355,8 @@ def qkv_proj(x: torch.Tensor, w_qkv: torch.Tensor, B: int, N: int, H: int, d: in
     _like("q", q, (B, N, H, 2, d), torch.bfloat16)
     _like("k", k, (B, N, H, 2, d), torch.bfloat16)
     _like("v", v, (B, N, H, 2 * d), torch.bfloat16)
-    _dev(x, w_qkv, q, k, v, *(() if rope is None else (rope,)))
-    _check("diffattn_qkv_proj", lib().diffattn_qkv_proj(
-        _ptr(x), _ptr(w_qkv), B, N, dm, H, d, _ptr(rope) if rope is not None else None, _ptr(q), _ptr(k), _ptr(v),
-        _stream()))
+    _launch("diffattn_qkv_proj", (x, w_qkv, q, k, v, *(() if rope is None else (rope,))),
+            _ptr(x), _ptr(w_qkv), B, N, dm, H, d, _ptr(rope) if rope is not None else None, _ptr(q), _ptr(k), _ptr(v))
     return q, k, v
 
 
@@ -369,8 +369,8 @@ def out_proj(o: torch.Tensor, w_o: torch.Tensor, out: torch.Tensor | None = None
     if out is None:
         out = torch.empty((M, n_out), dtype=torch.bfloat16, device=o.device)
     _like("out", out, (M, n_out), torch.bfloat16)
-    _dev(o, w_o, out)
-    _check("diffattn_out_proj", lib().diffattn_out_proj(_ptr(o), _ptr(w_o), M, K, n_out, _ptr(out), _stream()))
+    _launch("diffattn_out_proj", (o, w_o, out),
+            _ptr(o), _ptr(w_o), M, K, n_out, _ptr(out))
     return out
 
 
@@ -382,8 +382,8 @@ def diffattn_lambda_bwd(lq1: torch.Tensor, lk1: torch.Tensor, lq2: torch.Tensor,
     _scalar_f32("dlam", dlam)
     _dev(lq1, lk1, lq2, lk2, dlam)
     outs = [torch.empty_like(t) for t in (lq1, lk1, lq2, lk2)]
-    _check("diffattn_lambda_bwd", lib().diffattn_lambda_bwd(
-        _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), lq1.numel(), _ptr(dlam), *[_ptr(t) for t in outs], _stream()))
+    _launch("diffattn_lambda_bwd", (lq1, lk1, lq2, lk2, dlam, *outs),
+            _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), lq1.numel(), _ptr(dlam), *[_ptr(t) for t in outs])
     return tuple(outs)
 
 
@@ -420,17 +420,15 @@ def diffattn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
     if out is None:
         out = torch.empty((S, H, 2 * d), dtype=q.dtype, device=q.device)
     _like("out", out, (S, H, 2 * d), q.dtype)
-    _dev(workspace, out)
+    ts = (q, k_cache, v_cache, cu_seqlens, lam, rms_w, workspace, out)
+    ws_bytes = workspace.numel() * workspace.element_size()
     if mode == MODE_DIFF:
-        _check("diffattn_decode", lib().diffattn_decode(
-            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
-            _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _ptr(workspace), workspace.numel() * workspace.element_size(),
-            _stream()))
+        _launch("diffattn_decode", ts, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen),
+                _ptr(out), S, H, d, _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _ptr(workspace), ws_bytes)
     else:
-        _check("diffattn_decode_mode", lib().diffattn_decode_mode(
-            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
-            _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), int(mode), _ptr(workspace), workspace.numel() * workspace.element_size(),
-            _stream()))
+        _launch("diffattn_decode_mode", ts, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens),
+                int(max_seqlen), _ptr(out), S, H, d, _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps),
+                int(mode), _ptr(workspace), ws_bytes)
     return out
 
 
@@ -450,10 +448,9 @@ def diffattn_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
     if out is None:
         out = torch.empty((S, H, 2 * d), dtype=q.dtype, device=q.device)
     _like("out", out, (S, H, 2 * d), q.dtype)
-    _dev(out)
-    _check("diffattn_decode_noalloc", lib().diffattn_decode_noalloc(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
-        _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps), _stream()))
+    _launch("diffattn_decode_noalloc", (q, k_cache, v_cache, cu_seqlens, lam, rms_w, out),
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens), int(max_seqlen), _ptr(out), S, H, d,
+            _ptr(lam), float(lambda_init), _ptr(rms_w), float(eps))
     return out
 
 

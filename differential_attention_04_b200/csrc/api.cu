@@ -18,7 +18,11 @@ namespace {
 __device__ int g_status_word = 0;
 
 constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {};
+struct StatusSlot {
+  int* ptr;
+  unsigned long long ctx;  // context the address belongs to
+};
+StatusSlot g_status_slot[kMaxDevices] = {};
 std::mutex g_mu;
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
 
@@ -26,20 +30,25 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? DIFFATTN_OK : DIFFATTN_ERR_CUDA; }
 
-// Address of this device's status word (looked up once per device).
+// Address of this device's status word: looked up on the first call in each
+// context of the device (again after a cudaDeviceReset), or on every call when
+// the context id cannot be read.
 cudaError_t status_ptr(int** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_status_ptr[dev]) {
+  StatusSlot& slot = g_status_slot[dev];
+  if (!slot.ptr || ctx == 0 || slot.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_status_word);
     if (e != cudaSuccess) return e;
-    g_status_ptr[dev] = static_cast<int*>(p);
+    slot.ptr = static_cast<int*>(p);
+    slot.ctx = ctx;
   }
-  *out = g_status_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 
@@ -189,6 +198,32 @@ int bwd_tc_impl(const void* q, const void* k, const void* v, const void* dy, int
                                       dlambda, drms_w, workspace, saved, ctl, stream));
 }
 }  // namespace
+
+unsigned long long current_context_id() {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 }  // namespace diffattn
 
 using namespace diffattn;

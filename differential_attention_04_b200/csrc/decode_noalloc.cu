@@ -13,7 +13,10 @@
 // The array is a `static __device__` symbol.  In host code its name is only a
 // host-side stand-in, not a device address, so the host looks up the real
 // address once per device with cudaGetSymbolAddress (with that device
-// current) and passes it to the kernels.
+// current) and passes it to the kernels.  The cached address is tied to the
+// device's context: after a cudaDeviceReset the runtime creates a new context
+// (with a new id), and the next call looks the address up again instead of
+// handing the kernels an address of the old one.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -31,24 +34,32 @@ constexpr size_t kScratchBytes = DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_dev_ptr[kMaxDevices] = {};
+struct ScratchSlot {
+  void* ptr;
+  unsigned long long ctx;  // id of the context the address belongs to
+};
+ScratchSlot g_scratch_slot[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of g_decode_scratch on the current device (looked up on the
-// first call per device).
+// Device address of g_decode_scratch on the current device: looked up on the
+// first call per device (and again once the device's context has changed, or
+// on every call when the context id cannot be read).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = diffattn::current_context_id();
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_dev_ptr[dev]) {
+  ScratchSlot& slot = g_scratch_slot[dev];
+  if (!slot.ptr || ctx == 0 || slot.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_dev_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx = ctx;
   }
-  *out = g_scratch_dev_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 

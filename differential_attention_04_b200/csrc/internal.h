@@ -8,6 +8,12 @@
 
 namespace diffattn {
 
+// Unique id of the calling thread's current CUDA context (cuCtxGetId), or 0
+// when it cannot be read.  A context that cudaDeviceReset tore down and the
+// runtime re-created gets a new id, so per-device caches of device addresses
+// key on it and look the address up again.
+unsigned long long current_context_id();
+
 // Where kernels record a failed bounded wait, and how long a wait may spin.
 struct DevCtl {
   int* status;

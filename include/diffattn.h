@@ -24,6 +24,9 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never frees or keeps them.  The library allocates no device memory: the
  *    decode path takes a caller-provided workspace.
+ *  - Every pointer of a call must belong to the CURRENT device (the one
+ *    cudaSetDevice last selected on the calling thread), and `stream` must be
+ *    a stream of that device: the library launches on the current device.
  *  - Every call is asynchronous and ordered on `stream` (0 = legacy default
  *    stream).  The return value reports argument validation and launch
  *    errors only; nothing is synchronised.  A kernel-side failure (a bounded
@@ -403,7 +406,9 @@ int diffattn_decode_mode(const void* q, const void* k_cache, const void* v_cache
  *    S * H * ceil(max_seqlen / 512) must stay <= 8128 at d = 128).
  *  - Set-up: the first call on each device looks up the array's device
  *    address (cudaGetSymbolAddress, with that device current).  Make that
- *    first call before any stream capture.
+ *    first call before any stream capture.  The address is kept per device
+ *    and context: after cudaDeviceReset the next call (again before any
+ *    capture) looks it up in the new context.
  *  - Sharing: every call on a device uses the same array, which keeps the
  *    last call's contents.  Two calls that overlap on the GPU (on different
  *    streams, or from different host threads) race on it; the caller must

@@ -127,3 +127,29 @@ def test_bad_arguments_are_named(pre):
              dec.max_seqlen, lam, 0.5, dec.rms_w)
     _rejects("cu_seqlens", api.diffattn_decode_noalloc, dec.q, dec.k_cache, dec.v_cache, dec.cu_seqlens.long(),
              dec.max_seqlen, lam, 0.5, dec.rms_w)
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor on a given device: only what the binding's device check reads."""
+
+    is_cuda = True
+
+    def __init__(self, index: int):
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_tensors_on_two_devices_are_rejected_before_any_launch(monkeypatch):
+    # the library would launch on whichever device is current; tensors that
+    # live on two devices must never reach it
+    def no_launch(*a, **k):
+        raise AssertionError("the library was reached")
+
+    monkeypatch.setattr(api, "lib", no_launch)
+    with pytest.raises(ValueError, match="one device"):
+        api._dev(_FakeCuda(0), _FakeCuda(0), _FakeCuda(1))
+    with pytest.raises(ValueError, match="one device"):
+        api._launch("diffattn_fwd", (_FakeCuda(1), _FakeCuda(0)), 0)
+    assert api._dev(_FakeCuda(1), _FakeCuda(1)) == torch.device("cuda", 1)

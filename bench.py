@@ -597,6 +597,15 @@ def bench_small_prefill(api, wl, dev, reduce_max, barrier, rank, K=400):
             L.diffattn_fwd(*args)
         host_us.append((time.perf_counter() - t) / (K // 5) * 1e6)
         torch.cuda.synchronize()
+    # the same call with N = 0 passes every argument check and returns before any
+    # tensor map or launch: the cost of ctypes marshalling and validation alone
+    args0 = args[:6] + (0,) + args[7:]
+    floor_us = []
+    for _ in range(5):
+        t = time.perf_counter()
+        for _ in range(K // 5):
+            L.diffattn_fwd(*args0)
+        floor_us.append((time.perf_counter() - t) / (K // 5) * 1e6)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(K):
@@ -605,10 +614,15 @@ def bench_small_prefill(api, wl, dev, reduce_max, barrier, rank, K=400):
     torch.cuda.synchronize()
     dev_ms = reduce_max(a.elapsed_time(b)) / K
     flops_alg = prefill_flops(B, N, H, d, True, "algorithmic")
+    host = statistics.median(host_us)
+    floor = statistics.median(floor_us)
     return {"workload": f"B={B} N={N} H={H} d={d} causal bf16 (latency-bound)",
-            "host_us_per_call": statistics.median(host_us), "host_us_per_call_all": host_us,
+            "host_us_per_call": host, "host_us_per_call_all": host_us,
+            "ctypes_and_checks_us": floor, "library_launch_us": host - floor,
             "device_ms_per_launch": dev_ms, "achieved_tflops_algorithmic": flops_alg / (dev_ms * 1e-3) / 1e12,
             "how": "host: wall time of back-to-back diffattn_fwd calls through ctypes, no synchronisation inside; "
+                   "ctypes_and_checks_us: the same with N = 0 (validation only, no tensor map, no launch); "
+                   "library_launch_us: the difference (tensor-map lookup, launch); "
                    "device: CUDA events around K back-to-back launches",
             "gpu_launches": K + 20 + K}
 
@@ -846,6 +860,9 @@ def run_ours(args):
         line["qk4"] = bench_lowbit(api, inp, lam, y, peaks, peak_src, reduce_max, barrier, max(50, K // 8), 4)
     if not args.no_decode:
         line["decode"] = bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world)
+        # one long sequence among short ones: the grid must follow the real work
+        line["decode_skewed"] = bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world,
+                                             steps=50, seqlens=[32768] + [1024] * 63)
     del inp, y
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_inp = wl.make_prefill_case(args.workload, seed=1234, device="cpu")
@@ -858,10 +875,19 @@ def run_ours(args):
     return 0
 
 
-def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world, steps=20):
+def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world, steps=20, seqlens=None):
+    """The decode kernel pair on the KV-cache workload (64 sequences x 12 heads,
+    lengths ~ U{1024..32768}), or on the given sequence lengths."""
     import torch
 
-    inp = wl.make_decode_case(DECODE_WORKLOAD, seed=rank_seed(4321, rank), device=dev)
+    if seqlens is None:
+        inp = wl.make_decode_case(DECODE_WORKLOAD, seed=rank_seed(4321, rank), device=dev)
+        name = DECODE_WORKLOAD
+    else:
+        c = wl.DECODE_CASES[DECODE_WORKLOAD]
+        inp = wl.make_decode(len(seqlens), c["H"], c["d"], 0, 0, lambda_init=c["lambda_init"], w=c["w"],
+                             seed=rank_seed(4321, rank), device=dev, seqlens=seqlens)
+        name = f"skewed lengths ({seqlens[0]} then {len(seqlens) - 1} x {seqlens[1]})"
     S, H, _, d = inp.q.shape
     T = int(inp.seqlens.sum())
     lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
@@ -894,7 +920,7 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world
     traffic = read_profile_traffic("decode_decode_64x12")
     return {
         "metric": "decode HBM GB/s", "value": job_throughput(alg, world, ms) / 1e9, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
-        "workload": f"{DECODE_WORKLOAD}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
+        "workload": f"{name}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
                     f"({kv_bytes / 1e9:.2f} GB per step)",
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, **spec_fracs(gbs, "GB/s"),

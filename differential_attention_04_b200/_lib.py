@@ -10,8 +10,11 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdiffattn.so")
+# the bounds-checked build (same entry points; kernels record DIFFATTN_ERR_BOUNDS)
+DEBUG_LIB_PATH = os.path.join(_HERE, "libdiffattn_debug.so")
 
-_lib = None
+_handles = {}
+_active = LIB_PATH
 
 # name -> (restype, argtypes); mirrors include/diffattn.h
 _c_int, _c_float, _c_size, _vp, _c_ll = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_longlong
@@ -55,17 +58,30 @@ SIGNATURES = {
 }
 
 
-def lib() -> ctypes.CDLL:
-    """Load (once) and return the library with typed entry points."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
+def _load(path: str) -> ctypes.CDLL:
+    if path not in _handles:
+        if not os.path.exists(path):
             raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m differential_attention_04_b200.build`")
-        handle = ctypes.CDLL(LIB_PATH)
+                f"{path} is missing: build it with `python -m differential_attention_04_b200.build`"
+                + (" --debug" if path == DEBUG_LIB_PATH else ""))
+        handle = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(handle, name)
             fn.restype = res
             fn.argtypes = args
-        _lib = handle
-    return _lib
+        _handles[path] = handle
+    return _handles[path]
+
+
+def lib() -> ctypes.CDLL:
+    """Load (once) and return the active library with typed entry points."""
+    return _load(_active)
+
+
+def use_debug_library(on: bool = True) -> None:
+    """Route every binding call to the bounds-checked build (on) or back to the release one.
+
+    The two are separate libraries, each with its own device status word."""
+    global _active
+    _active = DEBUG_LIB_PATH if on else LIB_PATH
+    _load(_active)

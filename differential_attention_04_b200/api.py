@@ -12,7 +12,7 @@ import torch
 
 from ._lib import lib
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_BOUNDS = range(7)
 F32, BF16 = 0, 1
 # how the two maps are combined: softmax(S1) + c softmax(S2), c = -lambda, 0, +lambda
 MODE_DIFF, MODE_LAMBDA_ZERO, MODE_SUM = 0, 1, 2

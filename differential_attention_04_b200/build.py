@@ -3,7 +3,11 @@
 Each ``csrc/*.cu`` is compiled by nvcc into ``_build/`` (in parallel), then
 linked into ``differential_attention_04_b200/libdiffattn.so``.  Run as
 ``python -m differential_attention_04_b200.build``; ``--verbose-ptxas`` prints
-register / shared-memory usage per kernel.
+register / shared-memory usage per kernel.  ``--debug`` builds the
+bounds-checked variant instead (``-DDIFFATTN_DEBUG``, objects in
+``_build_debug/``, library ``libdiffattn_debug.so``): its kernels check every
+global index and tensor-map coordinate, skip an access out of range and
+record DIFFATTN_ERR_BOUNDS in the status word.
 """
 from __future__ import annotations
 
@@ -21,6 +25,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdiffattn.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libdiffattn_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -40,17 +46,20 @@ def _needs_build(obj: str, src: str) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose_ptxas: bool = False, force: bool = False) -> str:
+def build(verbose_ptxas: bool = False, force: bool = False, debug: bool = False) -> str:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    bdir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    os.makedirs(bdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
                     "--expt-relaxed-constexpr"]
+    if debug:
+        flags += ["-DDIFFATTN_DEBUG"]
     if verbose_ptxas:
         flags += ["-Xptxas", "-v"]
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
+        obj = os.path.join(bdir, os.path.basename(src).replace(".cu", ".o"))
         if force or verbose_ptxas or _needs_build(obj, src):
             cmd = [nvcc, "-c", src, "-o", obj] + flags
             r = subprocess.run(cmd, capture_output=True, text=True)
@@ -62,20 +71,21 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + ".tmp"
+    if force or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        tmp = lib + ".tmp"
         cmd = [nvcc, "-shared", "-o", tmp] + objs + ARCH + ["-Xcompiler", "-fPIC"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--verbose-ptxas", action="store_true")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="the bounds-checked library")
     a = ap.parse_args()
-    print(build(a.verbose_ptxas, a.force))
+    print(build(a.verbose_ptxas, a.force, a.debug))

@@ -69,39 +69,87 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps, kept per (base address, dims, element type, box): a
+// map is a pure function of those, so a cached one is valid whenever they
+// match (even for a new allocation that reuses the address).  A small table
+// with least-recently-used replacement keeps the host cost of a repeated call
+// to a lookup instead of a driver call per map.
+struct MapKey {
+  const void* base;
+  uint64_t d[4];
+  int kind;      // 1: uint8, 2: bf16, 4: packed e2m1
+  int box_rows;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && d[0] == o.d[0] && d[1] == o.d[1] && d[2] == o.d[2] && d[3] == o.d[3] &&
+           kind == o.kind && box_rows == o.box_rows;
+  }
+};
+struct MapSlot {
+  MapKey key;
+  CUtensorMap map;
+  unsigned long long used;  // 0: empty
+};
+constexpr int kMapSlots = 64;
+MapSlot g_map_slots[kMapSlots];
+unsigned long long g_map_clock = 0;
+std::mutex g_map_mu;
+
+bool encode_uncached(CUtensorMap* m, const MapKey& k) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {k.d[0], k.d[1], k.d[2], k.d[3]};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (k.kind == 4) {
+    // packed e2m1 codes: d0 codes (two per byte; d0 a multiple of 128); box =
+    // 128 codes x 1 x 128 rows x 1, widened to 128 bytes a row in shared
+    // memory (8 bytes of codes, then 8 bytes of gap, per 16 codes)
+    const cuuint64_t strides[3] = {k.d[0] / 2, k.d[0] / 2 * k.d[1], k.d[0] / 2 * k.d[1] * k.d[2]};
+    const cuuint32_t box[4] = {128, 1, 128, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void*>(k.base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  const uint64_t e = static_cast<uint64_t>(k.kind);
+  const cuuint64_t strides[3] = {k.d[0] * e, k.d[0] * k.d[1] * e, k.d[0] * k.d[1] * k.d[2] * e};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / e), 1, static_cast<cuuint32_t>(k.box_rows), 1};
+  return fn(m, e == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+            const_cast<void*>(k.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_cached(CUtensorMap* m, const MapKey& k) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapSlot* victim = &g_map_slots[0];
+  for (MapSlot& s : g_map_slots) {
+    if (s.used && s.key == k) {
+      s.used = ++g_map_clock;
+      *m = s.map;
+      return true;
+    }
+    if (s.used < victim->used) victim = &s;
+  }
+  if (!encode_uncached(m, k)) return false;
+  victim->key = k;
+  victim->map = *m;
+  victim->used = ++g_map_clock;
+  return true;
+}
+
 // 4-D map over a row-major tensor with dims (innermost first) d0..d3 of bf16
 // (esize 2) or byte (esize 1) elements; box = 128 bytes x 1 x box_rows x 1,
 // 128-byte swizzle, zero fill out of bounds.
 bool encode_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
                int esize = 2, int box_rows = 128) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const uint64_t e = static_cast<uint64_t>(esize);
-  const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {d0 * e, d0 * d1 * e, d0 * d1 * d2 * e};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 1, static_cast<cuuint32_t>(box_rows), 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
-            const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_cached(m, MapKey{base, {d0, d1, d2, d3}, esize, box_rows});
 }
 
 // 4-D map over packed e2m1 codes, dims (innermost first) d0 codes (two per
 // byte; d0 a multiple of 128), d1..d3; box = 128 codes x 1 x 128 rows x 1,
-// widened to 128 bytes a row in shared memory (8 bytes of codes, then 8 bytes
-// of gap, per 16 codes), 128-byte swizzle, zero fill out of bounds.  The base
-// must be 32-byte aligned and every stride a multiple of 32 bytes.
+// widened to 128 bytes a row in shared memory.  The base must be 32-byte
+// aligned and every stride a multiple of 32 bytes.
 bool encode_4d_e2m1(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {d0 / 2, d0 / 2 * d1, d0 / 2 * d1 * d2};
-  const cuuint32_t box[4] = {128, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_cached(m, MapKey{base, {d0, d1, d2, d3}, 4, 128});
 }
 
 bool fits_i32(long long x) { return x >= 0 && x < (1ll << 31); }
@@ -134,18 +182,17 @@ int fwd_lowbit_impl(int bits, const void* q_codes, const float* q_scales, const 
   if (bits == 4 && (!aligned32(q_codes) || !aligned32(k_codes))) return DIFFATTN_ERR_INVALID_ARG;
   if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   const bool codes_ok = bits == 4 ? encode_4d_e2m1(&tq, q_codes, d, 2ull * H, N, B) &&
                                         encode_4d_e2m1(&tk, k_codes, d, 2ull * H, N, B)
                                   : encode_4d(&tq, q_codes, d, 2ull * H, N, B, 1) &&
                                         encode_4d(&tk, k_codes, d, 2ull * H, N, B, 1);
-  if (!codes_ok || !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
-    return DIFFATTN_ERR_CUDA;
+  if (!codes_ok || !encode_4d(&tv, v, 2ull * d, H, N, B)) return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   cudaError_t e = status_ptr(&ctl.status);
   if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
-  return cuda_status(launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
+  return cuda_status(launch_prefill_sm100(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
                                           mode, q_scales, k_scales, bits, ctl, stream));
 }
 
@@ -199,6 +246,11 @@ int bwd_tc_impl(const void* q, const void* k, const void* v, const void* dy, int
 }
 }  // namespace
 
+int* status_word() {
+  int* p = nullptr;
+  return status_ptr(&p) == cudaSuccess ? p : nullptr;
+}
+
 unsigned long long current_context_id() {
   typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
   typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
@@ -240,6 +292,7 @@ const char* diffattn_status_string(int s) {
     case DIFFATTN_ERR_CUDA: return "CUDA error";
     case DIFFATTN_ERR_TIMEOUT: return "a kernel wait timed out";
     case DIFFATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case DIFFATTN_ERR_BOUNDS: return "an index was out of range (debug build; the access was skipped)";
     default: return "unknown status";
   }
 }
@@ -294,16 +347,16 @@ int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o, int 
                                                causal, lambda, lambda_init, rms_w, eps, mode, stream));
   }
   if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
-      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
+      !encode_4d(&tv, v, 2ull * d, H, N, B))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   cudaError_t e = status_ptr(&ctl.status);
   if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
   return cuda_status(
-      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, nullptr,
+      launch_prefill_sm100(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, nullptr,
                            nullptr, 16, ctl, stream));
 }
 
@@ -390,15 +443,15 @@ int diffattn_fwd_train(const void* q, const void* k, const void* v, void* o, int
   if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
   const BwdTcLayout L = bwd_tc_layout(B, N, H, d);
   if (!workspace || ws_bytes < L.bytes || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
-      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
+      !encode_4d(&tv, v, 2ull * d, H, N, B))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
   char* ws = static_cast<char*>(workspace);
-  return cuda_status(launch_prefill_sm100_stats(tq, tk, tv, &to, o, B, N, H, d, causal, lambda, lambda_init, rms_w,
+  return cuda_status(launch_prefill_sm100_stats(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w,
                                                 eps, mode, reinterpret_cast<float*>(ws + L.off_omaps),
                                                 reinterpret_cast<float*>(ws + L.off_stats), L.n_pad, ctl, stream));
 }

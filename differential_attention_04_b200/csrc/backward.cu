@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace diffattn {
@@ -55,7 +56,8 @@ __device__ __forceinline__ float warp_max(float x) {
 }
 
 struct BwdArgs {
-  int N, H, d, causal;
+  int B, N, H, d, causal;
+  int* dbg;           // debug builds: where the bounds checks record DIFFATTN_ERR_BOUNDS
   float dcoef;        // dc/dlambda of map 2's coefficient c (c itself is formed on the device from lambda)
   float lambda_init, eps;
   const float* rms_w;
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const T* __restrict__ q, 
     for (int u = 0; u < kMaxU; ++u) {
       const int c = lane + 32 * u;
       const float Gc = g * r * wv[u] * dyv[u] - O[u] * corr;
-      if (c < dv) a.G[row * dv + c] = Gc;
+      if (c < dv && DA_CHECK(a.dbg, row < static_cast<size_t>(a.B) * a.N * a.H)) a.G[row * dv + c] = Gc;
       d1 = fmaf(Gc, on1[u], d1);
       d2 = fmaf(Gc, on2[u], d2);
       dw_acc[u] = fmaf(g * r * O[u], dyv[u], dw_acc[u]);
@@ -379,6 +381,7 @@ __global__ void __launch_bounds__(256) bwd_keys_kernel(const T* __restrict__ q, 
     const int kj = kw + kk;
     if (kj >= N) continue;
     const size_t row = (static_cast<size_t>(b) * N + kj) * H + h;
+    if (!DA_CHECK(a.dbg, row < static_cast<size_t>(a.B) * N * H)) continue;  // debug builds
 #pragma unroll
     for (int u = 0; u < kMaxD; ++u) {
       const int c = lane + 32 * u;
@@ -513,6 +516,7 @@ __global__ void __launch_bounds__(256) bwd_queries_kernel(const T* __restrict__ 
     const int qi = qw + rr;
     if (qi >= N) continue;
     const size_t row = (static_cast<size_t>(b) * N + qi) * H + h;
+    if (!DA_CHECK(a.dbg, row < static_cast<size_t>(a.B) * N * H)) continue;  // debug builds
 #pragma unroll
     for (int u = 0; u < kMaxD; ++u) {
       const int c = lane + 32 * u;
@@ -556,6 +560,8 @@ cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const void
                          cudaStream_t stream) {
   const int dvw = 2 * d;
   BwdArgs a;
+  a.B = B;
+  a.dbg = debug_status();
   a.N = N;
   a.H = H;
   a.d = d;

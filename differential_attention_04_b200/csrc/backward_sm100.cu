@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(kGradThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
+      // debug builds: the block's rows lie in the tensors
+      (void)DA_CHECK(p.status, b < p.B && h < p.H && row0 < N);
       mbar_arrive_expect_tx(&bars->r_full, C::R_BYTES);
 #pragma unroll
       for (int m = 0; m < 2; ++m)
@@ -202,7 +204,12 @@ __global__ void __launch_bounds__(kGradThreads, 1)
         const int st = t % C::STAGES;
         if (!mbar_wait(&bars->c_empty[st], ((t / C::STAGES) & 1) ^ 1, wc)) break;
         const int c0 = (c_begin + t) * NC;
-        mbar_arrive_expect_tx(&bars->c_full[st], C::C_BYTES + (C::COL_STATS ? C::ST_BYTES : 0));
+        // debug builds: the column tile starts inside the tensors, and its
+        // statistics (an untiled copy, which nothing else bounds) lie in the
+        // [B][H][n_pad] array; when they do not, they are not copied
+        (void)DA_CHECK(p.status, c0 < N);
+        const bool st_ok = !C::COL_STATS || DA_CHECK(p.status, c0 + NC <= p.n_pad && bh < p.B * p.H);
+        mbar_arrive_expect_tx(&bars->c_full[st], C::C_BYTES + (C::COL_STATS && st_ok ? C::ST_BYTES : 0));
         uint8_t* base = sC + st * C::C_BYTES;
 #pragma unroll
         for (int m = 0; m < 2; ++m)
@@ -212,7 +219,7 @@ __global__ void __launch_bounds__(kGradThreads, 1)
 #pragma unroll
         for (int blk = 0; blk < C::VGB; ++blk)
           tma_load_4d(base + C::C_QK + blk * C::CBOX, &t_cvg, &bars->c_full[st], blk * 64, h, c0, b);
-        if constexpr (C::COL_STATS)
+        if (C::COL_STATS && st_ok)
           bulk_load_g2s(sST + st * C::ST_BYTES, p.stats + static_cast<size_t>(bh) * p.n_pad + c0, C::ST_BYTES,
                         &bars->c_full[st]);
       }
@@ -386,7 +393,7 @@ __global__ void __launch_bounds__(kGradThreads, 1)
     // ------------------------------------------------------- epilogue --
     mbar_wait(&bars->acc_done, 0, wdrain);
     tc_fence_after();
-    const bool live = grow < N;
+    const bool live = grow < N && DA_CHECK(p.status, b < p.B && h < p.H);
     const float scale = (KIND == kGradV) ? 1.0f : rsqrtf(static_cast<float>(D));
     // dV row [2d], or both maps' rows [2][d]: 2d contiguous floats either way
     float* orow = p.out + ((static_cast<size_t>(b) * N + (live ? grow : 0)) * p.H + h) * C::DV;
@@ -424,7 +431,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__
                                                        const float* __restrict__ lambda_ptr, int mode, float dcoef,
                                                        float lambda_init, float eps, int B, int N, int H, int n_pad,
                                                        __nv_bfloat16* __restrict__ G, float4* __restrict__ stats,
-                                                       float* __restrict__ dlambda, float* __restrict__ drms_w) {
+                                                       float* __restrict__ dlambda, float* __restrict__ drms_w,
+                                                       int* dbg) {
   constexpr int DV = 2 * D;
   constexpr int E = DV / 32;  // columns per lane, contiguous
   __shared__ float s_dw[8][DV];
@@ -496,7 +504,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__
       d1 += __shfl_xor_sync(0xffffffffu, d1, s);
       d2 += __shfl_xor_sync(0xffffffffu, d2, s);
     }
-    if (lane == 0) {
+    if (lane == 0 && DA_CHECK(dbg, row / H / N < B)) {
       const long long hh = row % H, bn = row / H;
       const long long n = bn % N, bb = bn / N;
       float* sp = reinterpret_cast<float*>(stats + (bb * H + hh) * n_pad + n);
@@ -549,7 +557,7 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   if (e == cudaSuccess) e = cudaMemsetAsync(dlambda, 0, sizeof(float), stream);
   if (e != cudaSuccess) return e;
   if (!stats_ready) {
-    e = launch_prefill_sm100_stats(m.q128, m.k128, m.v128, nullptr, nullptr, B, N, H, D, causal, lambda, lambda_init,
+    e = launch_prefill_sm100_stats(m.q128, m.k128, m.v128, nullptr, B, N, H, D, causal, lambda, lambda_init,
                                    rms_w, eps, mode, o_maps, reinterpret_cast<float*>(stats), L.n_pad, ctl, stream);
     if (e != cudaSuccess) return e;
   }
@@ -559,7 +567,7 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   const float dcoef = mode == 0 ? -1.0f : (mode == 2 ? 1.0f : 0.0f);
   bwd_prep_kernel<D><<<grid, 256, 0, stream>>>(o_maps, static_cast<const __nv_bfloat16*>(dy), rms_w, lambda, mode,
                                                dcoef, lambda_init, eps, B, N, H, L.n_pad, G, stats, dlambda,
-                                               drms_w);
+                                               drms_w, debug_status());
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   GradParams prm = {};

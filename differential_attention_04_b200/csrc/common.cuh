@@ -32,6 +32,20 @@ __device__ __forceinline__ void record_timeout(const WaitCtl& w) {
   *w.abort = 1;
 }
 
+// Debug builds (-DDIFFATTN_DEBUG): DA_CHECK(status, cond) records
+// DIFFATTN_ERR_BOUNDS (6) in the status word when `cond` fails and returns
+// `cond`, so that the caller skips the access; it never traps.  Release
+// builds do not evaluate `cond` (the check is always true).
+#ifdef DIFFATTN_DEBUG
+__device__ __forceinline__ bool da_check(int* status, bool ok) {
+  if (!ok) atomicCAS(status, 0, 6);
+  return ok;
+}
+#define DA_CHECK(status, cond) (::diffattn::da_check((status), (cond)))
+#else
+#define DA_CHECK(status, cond) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -54,14 +68,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// How long (ns) one try_wait may keep a waiting thread suspended before it
+// returns to check the time limit and the abort flag.  A suspended thread
+// issues nothing, so a warp that waits long (a whole item) takes no issue
+// slots from the warps it shares a scheduler with; it wakes when the phase
+// completes.
+constexpr uint32_t kSuspendHintNs = 200000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -96,6 +117,13 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uin
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
       "l"(m), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Hint: bring a 4-D tile into L2 ahead of its load (no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* m, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(m), "r"(c0),
+               "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05 --
@@ -323,10 +351,10 @@ __device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t* bar, uint32_t pa
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "n"(kSuspendHintNs)
         : "memory");
     return ok != 0;
   };
@@ -430,8 +458,54 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Named barrier over `count` threads that also returns whether `pred` held
+// in every one of them: a decision the whole group takes the same way.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Asynchronous stores into another CTA's shared memory (addresses from
+// map_to_cta), each completing `bytes` of transaction count on an mbarrier of
+// that CTA (also a shared::cluster address).
+__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, float a, float b, float c, float d,
+                                            uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   dst_cluster),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar_cluster)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t dst_cluster, float a, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(dst_cluster),
+               "f"(a), "r"(bar_cluster)
+               : "memory");
+}
+
+// Per-warpgroup register budgets (all four warps of a warpgroup execute the
+// same instruction; the counts must fit the registers the block launched with).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // ------------------------------------------------------------------- math --

@@ -9,17 +9,23 @@
 //
 // The work is bandwidth-bound (1 KiB of K and V per key and head, about 1.5
 // flop per byte), so it runs on CUDA cores:
-//   * decode_partial_kernel: one CTA per (key chunk, head, sequence).  Each
-//     warp streams its keys with 16-byte non-allocating loads, 8 keys in
-//     flight per lane group; lane l holds elements [8l, 8l+8) of the 256-wide
-//     K row (lanes 0-15: map 1, lanes 16-31: map 2) and of the V row.  The 8
-//     partial dot products are reduced across 16 lanes with a transposing
-//     shuffle tree (8 shuffles for 8 keys), and each map keeps its own online
-//     softmax state in the log2 domain.  The 4 warps merge, and the CTA writes
-//     (m1, l1, m2, l2, o1[256], o2[256]) for its chunk to the workspace.
-//   * decode_combine_kernel: one CTA per (head, sequence) merges the chunks
-//     with the log-sum-exp rescale per map, forms o1/l1 - lambda o2/l2, and
-//     applies the RMSNorm and scale.
+//   * decode_plan_kernel: one CTA turns cu_seqlens into the chunk offsets of
+//     each sequence (ceil(L / 512) chunks of up to 512 keys, at least one),
+//     so that the next kernel visits only chunks that exist.
+//   * decode_partial_kernel: a persistent grid (as many CTAs as fit on the
+//     GPU at once, spread over the heads) walks the chunks with a fixed
+//     stride.  Each warp streams its keys with 16-byte non-allocating loads,
+//     8 keys in flight per lane group; lane l holds elements [8l, 8l+8) of
+//     the 256-wide K row (lanes 0-15: map 1, lanes 16-31: map 2) and of the V
+//     row.  The 8 partial dot products are reduced across 16 lanes with a
+//     transposing shuffle tree (8 shuffles for 8 keys), and each map keeps its
+//     own online softmax state in the log2 domain.  The 4 warps merge, and
+//     the CTA writes (m1, l1, m2, l2, o1[256], o2[256]) for its chunk.
+//   * decode_combine_kernel: one CTA per (head, sequence) merges the
+//     sequence's chunks with the log-sum-exp rescale per map, forms
+//     o1/l1 - lambda o2/l2, and applies the RMSNorm and scale.
+// Workspace: the chunk records (room for S * ceil(max_seqlen / 512) chunks
+// per head), then the S + 1 chunk offsets.
 #include <math.h>
 
 #include "common.cuh"
@@ -45,192 +51,265 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   f[6] = bf16lo_to_f32(u.w); f[7] = bf16hi_to_f32(u.w);
 }
 
+// Keys of sequence s (its first key in *lo).  Debug builds check that the
+// keys lie in the packed cache (offsets non-decreasing and ending at
+// cu_seqlens[S]), where a sequence outside it is skipped, and that there are
+// at most max_seqlen of them: a longer sequence is cut to its first
+// max_seqlen keys, as release builds always do, and flagged.
+__device__ __forceinline__ int seq_keys(const int* __restrict__ cu, int s, int S, int max_seqlen, int* dbg,
+                                        int* lo) {
+  *lo = cu[s];
+  const int hi = cu[s + 1];
+  if (!DA_CHECK(dbg, *lo >= 0 && hi >= *lo && hi <= cu[S])) return 0;
+  (void)DA_CHECK(dbg, hi - *lo <= max_seqlen);
+  return min(hi - *lo, max_seqlen);
+}
+
+// chunk_start[s] = chunks of the sequences before s; chunk_start[S] = all chunks.
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const int* __restrict__ cu_seqlens, int S,
+                                                           int max_seqlen, int* __restrict__ chunk_start,
+                                                           int* dbg) {
+  __shared__ int warp_sum[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < S; base += 1024) {
+    const int s = base + static_cast<int>(threadIdx.x);
+    int n = 0;
+    if (s < S) {
+      int lo;
+      const int L = seq_keys(cu_seqlens, s, S, max_seqlen, dbg, &lo);
+      n = max(1, (L + kChunk - 1) / kChunk);
+    }
+    // inclusive scan of n over the block: within each warp, then over the warps
+    int x = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_sum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sum[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += y;
+      }
+      warp_sum[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? warp_sum[warp - 1] : 0) + x - n;
+    if (s < S) chunk_start[s] = carry + before;
+    carry += warp_sum[31];
+    __syncthreads();  // warp_sum is rewritten by the next pass
+  }
+  if (threadIdx.x == 0) chunk_start[S] = carry;
+}
+
 __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
-    const int* __restrict__ cu_seqlens, int max_seqlen, int H, int max_chunks, float* __restrict__ ws) {
-  const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
-  const int lo = cu_seqlens[s];
-  const int L = min(cu_seqlens[s + 1] - lo, max_seqlen);
-  const int c0 = chunk * kChunk;
-  if (c0 >= L && !(chunk == 0)) return;
+    const int* __restrict__ cu_seqlens, int S, int max_seqlen, int H, const int* __restrict__ chunk_start,
+    float* __restrict__ ws, int* dbg) {
+  const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = lane >> 4;  // 0: map 1, 1: map 2
   const int hl = lane & 15;
-
-  // This lane's slice of q (map `half`, elements [8*hl, 8*hl + 8)), pre-scaled
-  // so that scores come out in log2 units: s * log2(e) / sqrt(d).
-  float qf[8];
-  {
-    const uint4 qu = *reinterpret_cast<const uint4*>(q + (static_cast<size_t>(s) * H + h) * kDV + 8 * lane);
-    bf16x8_to_f32(qu, qf);
-    const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qf[i] *= sc;
-  }
-
-  float m1 = -INFINITY, m2 = -INFINITY;  // running max per map (same in all lanes)
-  float lsum = 0.f;                      // this lane's share of its map's running sum
-  float o1[8], o2[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o1[i] = o2[i] = 0.f;
-
-  const size_t row_stride = static_cast<size_t>(H) * kDV;  // elements between consecutive keys
-  const int kbeg = c0 + warp * kKeysPerWarp;
-  const int kend = min(L, kbeg + kKeysPerWarp);
-  const __nv_bfloat16* kbase = kc + static_cast<size_t>(lo) * row_stride + static_cast<size_t>(h) * kDV + 8 * lane;
-  const __nv_bfloat16* vbase = vc + static_cast<size_t>(lo) * row_stride + static_cast<size_t>(h) * kDV + 8 * lane;
-
-  for (int k0 = kbeg; k0 < kend; k0 += kGroup) {
-    uint4 kr[kGroup], vr[kGroup];
-#pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
-      const int key = k0 + g;
-      if (key < kend) {
-        kr[g] = ldg_stream_v4(kbase + static_cast<size_t>(key) * row_stride);
-        vr[g] = ldg_stream_v4(vbase + static_cast<size_t>(key) * row_stride);
-      } else {
-        kr[g] = make_uint4(0, 0, 0, 0);
-        vr[g] = make_uint4(0, 0, 0, 0);
-      }
-    }
-    // partial dot products of this lane's 8 elements, one per key
-    float part[kGroup];
-#pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
-      float kf[8];
-      bf16x8_to_f32(kr[g], kf);
-      float a = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a = fmaf(qf[i], kf[i], a);
-      part[g] = a;
-    }
-    // Transposing reduction over the 16 lanes of each half-warp: after the
-    // xor-8, xor-4 and xor-2 steps lane hl holds key g = 4*b3 + 2*b2 + b1
-    // (bits of hl) summed over 8 lanes; the xor-1 step completes the sum.
-    const bool b3 = (hl >> 3) & 1, b2 = (hl >> 2) & 1, b1 = (hl >> 1) & 1;
-    float r4[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float keep = b3 ? part[4 + i] : part[i];
-      const float give = b3 ? part[i] : part[4 + i];
-      r4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
-    }
-    float r2[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float keep = b2 ? r4[2 + i] : r4[i];
-      const float give = b2 ? r4[i] : r4[2 + i];
-      r2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
-    }
-    float sc;
-    {
-      const float keep = b1 ? r2[1] : r2[0];
-      const float give = b1 ? r2[0] : r2[1];
-      sc = keep + __shfl_xor_sync(0xffffffffu, give, 2);
-    }
-    sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-    const int my_key = 4 * b3 + 2 * b2 + b1;  // lanes 2g and 2g+1 of each half hold key g
-    if (k0 + my_key >= kend) sc = -INFINITY;
-
-    // group max per map, shared with the other half
-    float mx = sc;
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float mx_other = __shfl_xor_sync(0xffffffffu, mx, 16);
-    const float gm1 = half ? mx_other : mx;
-    const float gm2 = half ? mx : mx_other;
-    const float mn1 = fmaxf(m1, gm1), mn2 = fmaxf(m2, gm2);
-    const float al1 = fast_exp2(m1 - mn1), al2 = fast_exp2(m2 - mn2);  // exp2(-inf) = 0
-    m1 = mn1;
-    m2 = mn2;
-    const float p = fast_exp2(sc - (half ? mn2 : mn1));  // 0 for masked keys
-    lsum = lsum * (half ? al2 : al1) + ((lane & 1) ? 0.f : p);
-
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      o1[i] *= al1;
-      o2[i] *= al2;
-    }
-#pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
-      const float p1 = __shfl_sync(0xffffffffu, p, 2 * g);
-      const float p2 = __shfl_sync(0xffffffffu, p, 16 + 2 * g);
-      float vf[8];
-      bf16x8_to_f32(vr[g], vf);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        o1[i] = fmaf(p1, vf[i], o1[i]);
-        o2[i] = fmaf(p2, vf[i], o2[i]);
-      }
-    }
-  }
-
-  // running sums per map: sum the lanes of each half
-  float l = lsum;
-  l += __shfl_xor_sync(0xffffffffu, l, 8);
-  l += __shfl_xor_sync(0xffffffffu, l, 4);
-  l += __shfl_xor_sync(0xffffffffu, l, 2);
-  l += __shfl_xor_sync(0xffffffffu, l, 1);
-  const float l_other = __shfl_xor_sync(0xffffffffu, l, 16);
-  const float l1 = half ? l_other : l, l2 = half ? l : l_other;
-
-  // merge the warps of the CTA
+  const int total = chunk_start[S];
   __shared__ float sm_m[kWarps][2], sm_l[kWarps][2];
   __shared__ float sm_o[kWarps][2][kDV];
-  if (lane == 0) {
-    sm_m[warp][0] = m1; sm_m[warp][1] = m2;
-    sm_l[warp][0] = l1; sm_l[warp][1] = l2;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    sm_o[warp][0][8 * lane + i] = o1[i];
-    sm_o[warp][1][8 * lane + i] = o2[i];
-  }
-  __syncthreads();
-  float* rec = ws + ((static_cast<size_t>(s) * H + h) * max_chunks + chunk) * kRecFloats;
-  for (int mp = 0; mp < 2; ++mp) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][mp]);
-    float f[kWarps];
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) f[w] = (M == -INFINITY) ? 0.f : fast_exp2(sm_m[w][mp] - M);
-    for (int c = threadIdx.x; c < kDV; c += blockDim.x) {
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) acc = fmaf(f[w], sm_o[w][mp][c], acc);
-      rec[4 + mp * kDV + c] = acc;
+
+  for (int c = blockIdx.x; c < total; c += gridDim.x) {
+    // the sequence of chunk c: the last s with chunk_start[s] <= c
+    int s = 0;
+    {
+      int hi = S - 1;
+      while (s < hi) {
+        const int m = (s + hi + 1) >> 1;
+        if (chunk_start[m] <= c) s = m;
+        else hi = m - 1;
+      }
     }
-    if (threadIdx.x == 0) {
-      float Ls = 0.f;
+    const int chunk = c - chunk_start[s];
+    int lo;
+    const int L = seq_keys(cu_seqlens, s, S, max_seqlen, dbg, &lo);
+    const int c0 = chunk * kChunk;
+
+    // This lane's slice of q (map `half`, elements [8*hl, 8*hl + 8)), pre-scaled
+    // so that scores come out in log2 units: s * log2(e) / sqrt(d).
+    float qf[8];
+    {
+      const uint4 qu = *reinterpret_cast<const uint4*>(q + (static_cast<size_t>(s) * H + h) * kDV + 8 * lane);
+      bf16x8_to_f32(qu, qf);
+      const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) Ls = fmaf(f[w], sm_l[w][mp], Ls);
-      rec[2 * mp] = M;
-      rec[2 * mp + 1] = Ls;
+      for (int i = 0; i < 8; ++i) qf[i] *= sc;
     }
+
+    float m1 = -INFINITY, m2 = -INFINITY;  // running max per map (same in all lanes)
+    float lsum = 0.f;                      // this lane's share of its map's running sum
+    float o1[8], o2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o1[i] = o2[i] = 0.f;
+
+    const size_t row_stride = static_cast<size_t>(H) * kDV;  // elements between consecutive keys
+    const int kbeg = c0 + warp * kKeysPerWarp;
+    const int kend = min(L, kbeg + kKeysPerWarp);
+    const __nv_bfloat16* kbase = kc + static_cast<size_t>(lo) * row_stride + static_cast<size_t>(h) * kDV + 8 * lane;
+    const __nv_bfloat16* vbase = vc + static_cast<size_t>(lo) * row_stride + static_cast<size_t>(h) * kDV + 8 * lane;
+
+    for (int k0 = kbeg; k0 < kend; k0 += kGroup) {
+      uint4 kr[kGroup], vr[kGroup];
+#pragma unroll
+      for (int g = 0; g < kGroup; ++g) {
+        const int key = k0 + g;
+        if (key < kend) {
+          kr[g] = ldg_stream_v4(kbase + static_cast<size_t>(key) * row_stride);
+          vr[g] = ldg_stream_v4(vbase + static_cast<size_t>(key) * row_stride);
+        } else {
+          kr[g] = make_uint4(0, 0, 0, 0);
+          vr[g] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      // partial dot products of this lane's 8 elements, one per key
+      float part[kGroup];
+#pragma unroll
+      for (int g = 0; g < kGroup; ++g) {
+        float kf[8];
+        bf16x8_to_f32(kr[g], kf);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a = fmaf(qf[i], kf[i], a);
+        part[g] = a;
+      }
+      // Transposing reduction over the 16 lanes of each half-warp: after the
+      // xor-8, xor-4 and xor-2 steps lane hl holds key g = 4*b3 + 2*b2 + b1
+      // (bits of hl) summed over 8 lanes; the xor-1 step completes the sum.
+      const bool b3 = (hl >> 3) & 1, b2 = (hl >> 2) & 1, b1 = (hl >> 1) & 1;
+      float r4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float keep = b3 ? part[4 + i] : part[i];
+        const float give = b3 ? part[i] : part[4 + i];
+        r4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+      }
+      float r2[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float keep = b2 ? r4[2 + i] : r4[i];
+        const float give = b2 ? r4[i] : r4[2 + i];
+        r2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+      }
+      float sc;
+      {
+        const float keep = b1 ? r2[1] : r2[0];
+        const float give = b1 ? r2[0] : r2[1];
+        sc = keep + __shfl_xor_sync(0xffffffffu, give, 2);
+      }
+      sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+      const int my_key = 4 * b3 + 2 * b2 + b1;  // lanes 2g and 2g+1 of each half hold key g
+      if (k0 + my_key >= kend) sc = -INFINITY;
+
+      // group max per map, shared with the other half
+      float mx = sc;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mx_other = __shfl_xor_sync(0xffffffffu, mx, 16);
+      const float gm1 = half ? mx_other : mx;
+      const float gm2 = half ? mx : mx_other;
+      const float mn1 = fmaxf(m1, gm1), mn2 = fmaxf(m2, gm2);
+      const float al1 = fast_exp2(m1 - mn1), al2 = fast_exp2(m2 - mn2);  // exp2(-inf) = 0
+      m1 = mn1;
+      m2 = mn2;
+      const float p = fast_exp2(sc - (half ? mn2 : mn1));  // 0 for masked keys
+      lsum = lsum * (half ? al2 : al1) + ((lane & 1) ? 0.f : p);
+
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o1[i] *= al1;
+        o2[i] *= al2;
+      }
+#pragma unroll
+      for (int g = 0; g < kGroup; ++g) {
+        const float p1 = __shfl_sync(0xffffffffu, p, 2 * g);
+        const float p2 = __shfl_sync(0xffffffffu, p, 16 + 2 * g);
+        float vf[8];
+        bf16x8_to_f32(vr[g], vf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          o1[i] = fmaf(p1, vf[i], o1[i]);
+          o2[i] = fmaf(p2, vf[i], o2[i]);
+        }
+      }
+    }
+
+    // running sums per map: sum the lanes of each half
+    float l = lsum;
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    const float l_other = __shfl_xor_sync(0xffffffffu, l, 16);
+    const float l1 = half ? l_other : l, l2 = half ? l : l_other;
+
+    // merge the warps of the CTA
+    if (lane == 0) {
+      sm_m[warp][0] = m1; sm_m[warp][1] = m2;
+      sm_l[warp][0] = l1; sm_l[warp][1] = l2;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sm_o[warp][0][8 * lane + i] = o1[i];
+      sm_o[warp][1][8 * lane + i] = o2[i];
+    }
+    __syncthreads();
+    float* rec = ws + (static_cast<size_t>(c) * H + h) * kRecFloats;
+    for (int mp = 0; mp < 2; ++mp) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][mp]);
+      float f[kWarps];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) f[w] = (M == -INFINITY) ? 0.f : fast_exp2(sm_m[w][mp] - M);
+      for (int cc = threadIdx.x; cc < kDV; cc += blockDim.x) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) acc = fmaf(f[w], sm_o[w][mp][cc], acc);
+        rec[4 + mp * kDV + cc] = acc;
+      }
+      if (threadIdx.x == 0) {
+        float Ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) Ls = fmaf(f[w], sm_l[w][mp], Ls);
+        rec[2 * mp] = M;
+        rec[2 * mp + 1] = Ls;
+      }
+    }
+    __syncthreads();  // the merge buffers are refilled by the next chunk
   }
 }
 
 __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __restrict__ ws,
-                                                             const int* __restrict__ cu_seqlens, int max_seqlen,
-                                                             int H, int max_chunks, __nv_bfloat16* __restrict__ o,
+                                                             const int* __restrict__ chunk_start, int H,
+                                                             __nv_bfloat16* __restrict__ o,
                                                              const float* __restrict__ lambda_ptr, int mode,
                                                              float lambda_init, const float* __restrict__ rms_w,
-                                                             float eps) {
+                                                             float eps, int* dbg) {
   const int h = blockIdx.x, s = blockIdx.y;
   const int c = threadIdx.x;
-  const int L = min(cu_seqlens[s + 1] - cu_seqlens[s], max_seqlen);
-  const int nch = max(1, (L + kChunk - 1) / kChunk);
-  const float* rec0 = ws + (static_cast<size_t>(s) * H + h) * max_chunks * kRecFloats;
+  const int first = chunk_start[s];
+  int nch = chunk_start[s + 1] - first;
+  if (!DA_CHECK(dbg, nch >= 1 && first >= 0 && first + nch <= chunk_start[gridDim.y])) nch = 0;
   float M1 = -INFINITY, M2 = -INFINITY;
   for (int i = 0; i < nch; ++i) {
-    M1 = fmaxf(M1, rec0[i * kRecFloats + 0]);
-    M2 = fmaxf(M2, rec0[i * kRecFloats + 2]);
+    const float* r = ws + (static_cast<size_t>(first + i) * H + h) * kRecFloats;
+    M1 = fmaxf(M1, r[0]);
+    M2 = fmaxf(M2, r[2]);
   }
   float L1 = 0.f, L2 = 0.f, O1 = 0.f, O2 = 0.f;
   for (int i = 0; i < nch; ++i) {
-    const float* r = rec0 + i * kRecFloats;
+    const float* r = ws + (static_cast<size_t>(first + i) * H + h) * kRecFloats;
     const float f1 = fast_exp2(r[0] - M1), f2 = fast_exp2(r[2] - M2);
     L1 = fmaf(f1, r[1], L1);
     L2 = fmaf(f2, r[3], L2);
@@ -252,27 +331,58 @@ __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __rest
   o[(static_cast<size_t>(s) * H + h) * kDV + c] = __float2bfloat16_rn((1.0f - lambda_init) * rms_w[c] * ov * rs);
 }
 
+namespace {
+// Byte offset of the chunk offsets in the workspace (after the records).
+size_t plan_offset(int S, int H, int max_seqlen) {
+  const size_t chunks = (static_cast<size_t>(max_seqlen) + kChunk - 1) / kChunk;
+  const size_t rec = static_cast<size_t>(S) * chunks * H * kRecFloats * sizeof(float);
+  return (rec + 15) & ~static_cast<size_t>(15);
+}
+}  // namespace
+
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen) {
   if (S <= 0 || H <= 0 || d != kD || max_seqlen <= 0) return 0;
-  const size_t chunks = (static_cast<size_t>(max_seqlen) + kChunk - 1) / kChunk;
-  return static_cast<size_t>(S) * H * chunks * kRecFloats * sizeof(float);
+  return plan_offset(S, H, max_seqlen) + ((static_cast<size_t>(S + 1) * sizeof(int) + 15) & ~static_cast<size_t>(15));
 }
 
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
                           int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
                           const float* rms_w, float eps, int mode, void* workspace, cudaStream_t stream) {
   (void)d;
-  const int max_chunks = (max_seqlen + kChunk - 1) / kChunk;
-  dim3 grid(max_chunks, H, S);
-  decode_partial_kernel<<<grid, kWarps * 32, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
-      static_cast<const __nv_bfloat16*>(v_cache), cu_seqlens, max_seqlen, H, max_chunks,
-      static_cast<float*>(workspace));
-  cudaError_t e = cudaGetLastError();
+  int* dbg = debug_status();
+  // persistent partial grid: the CTAs that fit on the GPU at once, spread over
+  // the heads (looked up once per device)
+  static int resident[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<dim3(H, S), kDV, 0, stream>>>(static_cast<const float*>(workspace), cu_seqlens,
-                                                        max_seqlen, H, max_chunks, static_cast<__nv_bfloat16*>(o),
-                                                        lambda, mode, lambda_init, rms_w, eps);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (resident[dev] == 0) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_partial_kernel, kWarps * 32, 0);
+    if (e != cudaSuccess) return e;
+    resident[dev] = sms * (per_sm > 0 ? per_sm : 1);
+  }
+  const long long max_chunks = (static_cast<long long>(max_seqlen) + kChunk - 1) / kChunk;
+  const long long upper = static_cast<long long>(S) * max_chunks;  // chunks there can be
+  long long gx = resident[dev] / H;
+  if (gx < 1) gx = 1;
+  if (gx > upper) gx = upper;
+  if (gx > 0x7fffffffll) gx = 0x7fffffffll;
+  float* recs = static_cast<float*>(workspace);
+  int* chunk_start = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan_offset(S, H, max_seqlen));
+  decode_plan_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, S, max_seqlen, chunk_start, dbg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_partial_kernel<<<dim3(static_cast<unsigned>(gx), H), kWarps * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
+      static_cast<const __nv_bfloat16*>(v_cache), cu_seqlens, S, max_seqlen, H, chunk_start, recs, dbg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<<<dim3(H, S), kDV, 0, stream>>>(recs, chunk_start, H, static_cast<__nv_bfloat16*>(o), lambda,
+                                                        mode, lambda_init, rms_w, eps, dbg);
   return cudaGetLastError();
 }
 

@@ -14,6 +14,19 @@ namespace diffattn {
 // key on it and look the address up again.
 unsigned long long current_context_id();
 
+// Device address of the status word on the current device (nullptr when it
+// cannot be looked up).
+int* status_word();
+// What a kernel's debug bounds checks (DA_CHECK) record into: the status word
+// in a debug build, nullptr in a release build (where the checks compile away).
+inline int* debug_status() {
+#ifdef DIFFATTN_DEBUG
+  return status_word();
+#else
+  return nullptr;
+#endif
+}
+
 // Where kernels record a failed bounded wait, and how long a wait may spin.
 struct DevCtl {
   int* status;
@@ -35,11 +48,10 @@ __host__ __device__ inline float map2_coefficient(int mode, float lam) {
 
 // Tensor-core (tcgen05) prefill, d in {64, 128} for bf16 queries and keys,
 // d = 128 for low-bit ones (q_scale, k_scale non-null; qk_bits 8: e4m3 codes,
-// 4: packed e2m1 codes).  tq/tk map [B, N, H*2, d]; tv and to map
-// [B, N, H, 2d]; boxes are 128 bytes (bf16, e4m3) or 128 elements (e2m1) x
-// 128 rows with 128-byte swizzle.
-cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                 const CUtensorMap& to, void* o,
+// 4: packed e2m1 codes).  tq/tk map [B, N, H*2, d]; tv maps [B, N, H, 2d];
+// boxes are 128 bytes (bf16, e4m3) or 128 elements (e2m1) x 128 rows with
+// 128-byte swizzle.  The output o [B, N, H, 2d] (bf16) is written directly.
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, int mode, const float* q_scale,
                                  const float* k_scale, int qk_bits, DevCtl ctl, cudaStream_t stream);
@@ -80,9 +92,9 @@ cudaError_t launch_bwd_sm100(const BwdTcMaps& m, const void* dy, int B, int N, i
                              bool stats_ready, DevCtl ctl, cudaStream_t stream);
 // The tcgen05 prefill in its statistics mode: per map, O_i / l_i into
 // o_maps and the log2-sum-exp into component i of the float4 rows of lse;
-// with `to` (the output map over o) non-null, the normalised output too.
+// with o non-null, the normalised output too.
 cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                       const CUtensorMap* to, void* o, int B, int N, int H, int d, int causal,
+                                       void* o, int B, int N, int H, int d, int causal,
                                        const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                                        float* o_maps, float* lse, int n_pad, DevCtl ctl, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,

@@ -14,6 +14,7 @@
 // then every lane accumulates the output channels c = lane + 32u.
 #include <math.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace diffattn {
@@ -28,7 +29,7 @@ constexpr int kMaxU = 8;  // ceil(2 * 128 / 32)
 __global__ void __launch_bounds__(256) prefill_simt_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, float* __restrict__ o,
     int N, int H, int d, int causal, const float* __restrict__ lambda_ptr, float lambda_init,
-    const float* __restrict__ rms_w, float eps, int mode) {
+    const float* __restrict__ rms_w, float eps, int mode, int* dbg) {
   extern __shared__ float smem[];
   const int kstride = (d % 2 == 0) ? d + 1 : d;  // odd row pitch: conflict-free column reads
   const int dv = 2 * d;
@@ -163,7 +164,10 @@ __global__ void __launch_bounds__(256) prefill_simt_f32_kernel(
 #pragma unroll
     for (int u = 0; u < kMaxU; ++u) {
       const int c = lane + 32 * u;
-      if (c < dv) ob[static_cast<size_t>(qi) * tok_v + c] = out_scale * rms_w[c] * ov[u] * rs;
+      // debug builds: the element lies in o [B, N, H, 2d]
+      if (c < dv && DA_CHECK(dbg, (ob - o) + static_cast<size_t>(qi) * tok_v + c <
+                                      static_cast<size_t>(gridDim.z) * N * tok_v))
+        ob[static_cast<size_t>(qi) * tok_v + c] = out_scale * rms_w[c] * ov[u] * rs;
     }
   }
 }
@@ -179,7 +183,7 @@ cudaError_t launch_prefill_simt_f32(const float* q, const float* k, const float*
   if (e != cudaSuccess) return e;
   dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, H, B);
   prefill_simt_f32_kernel<<<grid, 256, smem, stream>>>(q, k, v, o, N, H, d, causal, lambda, lambda_init, rms_w,
-                                                       eps, mode);
+                                                       eps, mode, debug_status());
   return cudaGetLastError();
 }
 

@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
           if (leader) mbar_arrive_expect_tx(&bars->full[s], 2 * k2StageBytes);
           uint8_t* st = smem + s * k2StageBytes;
           const uint32_t fb = lead(&bars->full[s]);
+          // debug builds: the tiles start inside A [M, K] and B [N, K] (TMA fills the rest with zeros)
+          (void)DA_CHECK(p.status, ks * kPBK < p.K && tm * k2BM < p.M && tn * k2BN < p.N);
           tma_load_4d_pair(st, &ta, fb, ks * kPBK, 0, tm * k2BM + 128 * static_cast<int>(rank), 0);
           tma_load_4d_pair(st + k2ABytes, &tb, fb, ks * kPBK, 0, tn * k2BN + 128 * static_cast<int>(rank), 0);
         }
@@ -203,6 +205,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
             v[2 * j + 1] = __float_as_uint(fmaf(x0, t2.y, x1 * t2.x));
           }
         }
+        // debug builds: the 32 columns lie in their output, and their rotary entries in the table
+        if (!DA_CHECK(p.status, c_in >= 0 && c_in + 32 <= width && (!p.rope || col >= p.rope_end ||
+                                                                    pos < p.seq_len)))
+          continue;
         uint4* dst = reinterpret_cast<uint4*>(obase + static_cast<size_t>(m) * width + c_in);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
@@ -226,11 +232,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-__global__ void rope_table_kernel(int seq_len, int d, double base, float2* table) {
+__global__ void rope_table_kernel(int seq_len, int d, double base, float2* table, int* dbg) {
   const int half = d / 2;
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= static_cast<long long>(seq_len) * half) return;
   const int n = static_cast<int>(i / half), j = static_cast<int>(i % half);
+  if (!DA_CHECK(dbg, n < seq_len && j < half)) return;
   const double ang = static_cast<double>(n) * pow(base, -2.0 * j / d);
   double s, c;
   sincos(ang, &s, &c);
@@ -273,7 +280,7 @@ cudaError_t launch_proj_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const
 cudaError_t launch_rope_table(int seq_len, int d, double base, float* table, cudaStream_t stream) {
   const long long n = static_cast<long long>(seq_len) * (d / 2);
   const unsigned grid = static_cast<unsigned>((n + 255) / 256);
-  rope_table_kernel<<<grid, 256, 0, stream>>>(seq_len, d, base, reinterpret_cast<float2*>(table));
+  rope_table_kernel<<<grid, 256, 0, stream>>>(seq_len, d, base, reinterpret_cast<float2*>(table), debug_status());
   return cudaGetLastError();
 }
 

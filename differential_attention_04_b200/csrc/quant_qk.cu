@@ -28,6 +28,7 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace diffattn {
@@ -71,7 +72,9 @@ __device__ __forceinline__ Walk walk_of(int vec) {
 }
 
 __global__ void __launch_bounds__(kThreadsQ) qk_absmax_kernel(const __nv_bfloat16* __restrict__ x, int N, int H,
-                                                              int d, unsigned int* __restrict__ amax_bits) {
+                                                              int d, unsigned int* __restrict__ amax_bits,
+                                                              int* dbg) {
+  // debug builds: the elements read below lie in x [B, N, H, 2, d] (rows n0 .. n0 + rows - 1 of group g)
   const int g = blockIdx.y;
   const int b = g / (2 * H), hi = g % (2 * H);
   const int n0 = blockIdx.x * kTokPerCta;
@@ -80,7 +83,8 @@ __global__ void __launch_bounds__(kThreadsQ) qk_absmax_kernel(const __nv_bfloat1
   const Walk w = walk_of(vec);
   const size_t row_vecs = static_cast<size_t>(2 * H) * vec;  // vectors from one token row to the next
   float m = 0.f;
-  if (w.active) {
+  if (w.active && DA_CHECK(dbg, n0 >= 0 && rows >= 1 && n0 + rows <= N && b < static_cast<int>(gridDim.y) / (2 * H) &&
+                                    d % 8 == 0)) {
     for (int c = w.c0; c < vec; c += w.c_step) {
       const uint4* p = row_ptr(x, b, n0, hi, N, H, d) + c;
       for (int r = w.r0; r < rows; r += kUnroll * w.r_step) {
@@ -150,7 +154,7 @@ __device__ __forceinline__ uint32_t encode8_e2m1(const float (&r)[8]) {
 template <int BITS>
 __global__ void __launch_bounds__(kThreadsQ) qk_quant_kernel(const __nv_bfloat16* __restrict__ x, int N, int H,
                                                              int d, const float* __restrict__ scales,
-                                                             uint8_t* __restrict__ codes) {
+                                                             uint8_t* __restrict__ codes, int* dbg) {
   const int g = blockIdx.y;
   const int b = g / (2 * H), hi = g % (2 * H);
   const int n0 = blockIdx.x * kTokPerCta;
@@ -158,6 +162,10 @@ __global__ void __launch_bounds__(kThreadsQ) qk_quant_kernel(const __nv_bfloat16
   const int vec = d / 8;
   const Walk w = walk_of(vec);
   if (!w.active) return;
+  // debug builds: rows n0 .. n0 + rows - 1 of group g lie in x and in the codes
+  if (!DA_CHECK(dbg, n0 >= 0 && rows >= 1 && n0 + rows <= N && b < static_cast<int>(gridDim.y) / (2 * H) &&
+                         d % 8 == 0))
+    return;
   const float s = __ldg(scales + g);
   const size_t row_vecs = static_cast<size_t>(2 * H) * vec;
   constexpr int kOutBytes = BITS == 8 ? 8 : 4;  // code bytes per vector
@@ -199,12 +207,13 @@ cudaError_t launch_quantize_qk(const void* x, int B, int N, int H, int d, int bi
   if (e != cudaSuccess) return e;
   const dim3 grid((N + kTokPerCta - 1) / kTokPerCta, G);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  qk_absmax_kernel<<<grid, kThreadsQ, 0, stream>>>(xb, N, H, d, reinterpret_cast<unsigned int*>(scales));
+  int* dbg = debug_status();
+  qk_absmax_kernel<<<grid, kThreadsQ, 0, stream>>>(xb, N, H, d, reinterpret_cast<unsigned int*>(scales), dbg);
   qk_scale_kernel<<<(G + 255) / 256, 256, 0, stream>>>(scales, G, bits == 8 ? kE4m3Max : kE2m1Max);
   if (bits == 8)
-    qk_quant_kernel<8><<<grid, kThreadsQ, 0, stream>>>(xb, N, H, d, scales, static_cast<uint8_t*>(codes));
+    qk_quant_kernel<8><<<grid, kThreadsQ, 0, stream>>>(xb, N, H, d, scales, static_cast<uint8_t*>(codes), dbg);
   else
-    qk_quant_kernel<4><<<grid, kThreadsQ, 0, stream>>>(xb, N, H, d, scales, static_cast<uint8_t*>(codes));
+    qk_quant_kernel<4><<<grid, kThreadsQ, 0, stream>>>(xb, N, H, d, scales, static_cast<uint8_t*>(codes), dbg);
   return cudaGetLastError();
 }
 

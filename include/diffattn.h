@@ -35,6 +35,11 @@
  *  - Tensors are dense and row-major in the layouts given below; every
  *    tensor pointer must be 16-byte aligned.
  *  - Return values are diffattn_status codes; 0 is success.
+ *  - Debug build (libdiffattn_debug.so, compiled with -DDIFFATTN_DEBUG): the
+ *    same entry points, whose kernels also check every global index and
+ *    tensor-map coordinate before use.  An index out of range is skipped
+ *    (never trapped) and DIFFATTN_ERR_BOUNDS is recorded in the device status
+ *    word.  The release library compiles these checks away.
  */
 #ifndef DIFFATTN_H_
 #define DIFFATTN_H_
@@ -52,7 +57,9 @@ typedef enum {
   DIFFATTN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, d)      */
   DIFFATTN_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed         */
   DIFFATTN_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out           */
-  DIFFATTN_ERR_WORKSPACE = 5     /* workspace missing or too small            */
+  DIFFATTN_ERR_WORKSPACE = 5,    /* workspace missing or too small            */
+  DIFFATTN_ERR_BOUNDS = 6        /* debug build only: a kernel found an index
+                                    out of range and skipped the access       */
 } diffattn_status;
 
 typedef enum {
@@ -365,7 +372,12 @@ size_t diffattn_decode_workspace_size(int S, int H, int d, int max_seqlen);
  * Errors: DIFFATTN_ERR_INVALID_ARG, DIFFATTN_ERR_WORKSPACE,
  * DIFFATTN_ERR_CUDA.  A length outside [1, max_seqlen] is not detected on
  * the host (cu_seqlens lives on the device): the kernel skips keys beyond
- * max_seqlen and writes NaN for an empty sequence.
+ * max_seqlen and writes NaN for an empty sequence; the debug build also
+ * records DIFFATTN_ERR_BOUNDS for a length above max_seqlen, and skips a
+ * sequence whose offsets fall outside [0, cu_seqlens[S]].
+ * Work layout: a planning kernel turns cu_seqlens into each sequence's
+ * ceil(L / 512) key chunks, so the kernels visit only chunks that exist
+ * (a long sequence among short ones costs its own keys, not S times them).
  */
 int diffattn_decode(const void* q, const void* k_cache, const void* v_cache,
                     const int* cu_seqlens, int max_seqlen, void* o, int S,
@@ -402,8 +414,10 @@ int diffattn_decode_mode(const void* q, const void* k_cache, const void* v_cache
  *
  *  - Limit: problems with diffattn_decode_workspace_size(S, H, d,
  *    max_seqlen) > DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES are rejected with
- *    DIFFATTN_ERR_WORKSPACE before anything is launched (for example
- *    S * H * ceil(max_seqlen / 512) must stay <= 8128 at d = 128).
+ *    DIFFATTN_ERR_WORKSPACE before anything is launched (at d = 128 the size
+ *    is 2064 * S * H * ceil(max_seqlen / 512) bytes plus the S + 1 chunk
+ *    offsets, so S * H * ceil(max_seqlen / 512) must stay a little under
+ *    8128).
  *  - Set-up: the first call on each device looks up the array's device
  *    address (cudaGetSymbolAddress, with that device current).  Make that
  *    first call before any stream capture.  The address is kept per device
@@ -426,8 +440,8 @@ int diffattn_decode_noalloc(const void* q, const void* k_cache,
 
 /*
  * diffattn_device_status -- synchronises the current device, then returns
- * the device-side status word (DIFFATTN_OK or DIFFATTN_ERR_TIMEOUT) in
- * *status_out and clears it.  Returns DIFFATTN_ERR_CUDA if the device could
+ * the device-side status word (DIFFATTN_OK, DIFFATTN_ERR_TIMEOUT, or in the
+ * debug build DIFFATTN_ERR_BOUNDS) in *status_out and clears it.  Returns DIFFATTN_ERR_CUDA if the device could
  * not be queried.
  */
 int diffattn_device_status(int* status_out);

@@ -169,11 +169,16 @@ def test_validation_without_gpu(L):
 def test_workspace_size(L):
     assert L.diffattn_decode_workspace_size(0, 12, 128, 100) == 0
     assert L.diffattn_decode_workspace_size(4, 12, 64, 100) == 0
+    # one record per (key chunk of up to 512 keys, head): m1, l1, m2, l2 and two
+    # 256-wide partial outputs in float32, then the S + 1 chunk offsets (int32)
+    rec = (4 + 2 * 256) * 4
     one = L.diffattn_decode_workspace_size(1, 1, 128, 1)
-    assert one > 0 and one % 16 == 0
-    # grows with the number of key chunks per sequence and with S * H
-    assert L.diffattn_decode_workspace_size(3, 5, 128, 1) == 15 * one
-    assert L.diffattn_decode_workspace_size(1, 1, 128, 100000) > one
+    assert one % 16 == 0 and one >= rec + 2 * 4
+    many = L.diffattn_decode_workspace_size(3, 5, 128, 1)
+    assert many % 16 == 0 and many >= 15 * rec + 4 * 4
+    # grows with the number of key chunks per sequence
+    long = L.diffattn_decode_workspace_size(1, 1, 128, 100000)
+    assert long % 16 == 0 and long >= 196 * rec
 
 
 def test_wait_limit_setter(L):

@@ -107,13 +107,17 @@ def prefill_row_flops(N, d, causal, convention):
     return (16.0 if convention == "metric" else 12.0) * N * d * (0.5 if causal else 1.0)
 
 
-def read_profile_traffic(kernel_tag: str):
+def read_profile_traffic(kernel_tag: str, algorithmic_bytes=None):
     """Per-launch DRAM bytes from a committed ncu summary, if it matches the current kernel source.
 
     The summary names the sources it was captured on (`source_files:`, paths
     under csrc/, comma-separated; the prefill or decode kernel's file when
     absent) and their hash (`source_sha256_16`: sha256 of the files' bytes in
-    that order); a summary of older sources gives None."""
+    that order); a summary of older sources gives None.  Where the summary
+    states the algorithmic bytes of the launch its traffic describes
+    (`algorithmic_bytes_per_launch`, for kernels whose traffic follows their
+    algorithmic bytes) and the caller passes its own launch's, the traffic is
+    scaled by their ratio."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
@@ -134,8 +138,11 @@ def read_profile_traffic(kernel_tag: str):
     if vals.get("source_sha256_16") != h.hexdigest()[:16]:
         return None
     try:
-        return float(vals["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        traffic = float(vals["traffic_bytes_per_launch"])
+        if algorithmic_bytes is not None and "algorithmic_bytes_per_launch" in vals:
+            traffic *= algorithmic_bytes / float(vals["algorithmic_bytes_per_launch"])
+        return traffic
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
 
 
@@ -917,17 +924,17 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world
     io_bytes = S * H * 2 * d * 2 * 2
     alg = kv_bytes + io_bytes
     gbs = alg / (ms * 1e-3) / 1e9
-    traffic = read_profile_traffic("decode_decode_64x12")
+    traffic = read_profile_traffic("decode_decode_64x12", alg)
     return {
         "metric": "decode HBM GB/s", "value": job_throughput(alg, world, ms) / 1e9, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
         "workload": f"{name}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
                     f"({kv_bytes / 1e9:.2f} GB per step)",
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, **spec_fracs(gbs, "GB/s"),
-                     "kernel": "decode_partial_kernel + decode_combine_kernel",
+                     "kernel": "decode_plan_kernel + decode_partial_kernel + decode_combine_kernel",
                      "algorithmic_bytes": alg, "peak_source": f"{peak_src} HBM copy"},
         "clocks": clk, "loop_wall_s": wall,
-        "gpu_launches": 2 * steps,
+        "gpu_launches": 3 * steps,  # planning, partial and combine kernels
     }
 
 

@@ -32,24 +32,35 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? DIFFATTN_OK : DIFFATT
 
 // Address of this device's status word: looked up on the first call in each
 // context of the device (again after a cudaDeviceReset), or on every call when
-// the context id cannot be read.
-cudaError_t status_ptr(int** out) {
+// the context id cannot be read.  The device and context id are reported too
+// (dev, ctx may be null), so that a launcher need not look them up again.
+cudaError_t status_ptr(int** out, int* dev_out = nullptr, unsigned long long* ctx_out = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   const unsigned long long ctx = current_context_id();
-  std::lock_guard<std::mutex> lk(g_mu);
   StatusSlot& slot = g_status_slot[dev];
-  if (!slot.ptr || ctx == 0 || slot.ctx != ctx) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_status_word);
-    if (e != cudaSuccess) return e;
-    slot.ptr = static_cast<int*>(p);
-    slot.ctx = ctx;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!slot.ptr || ctx == 0 || slot.ctx != ctx) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_status_word);
+      if (e != cudaSuccess) return e;
+      slot.ptr = static_cast<int*>(p);
+      slot.ctx = ctx;
+    }
+    *out = slot.ptr;
   }
-  *out = slot.ptr;
+  if (dev_out) *dev_out = dev;
+  if (ctx_out) *ctx_out = ctx;
   return cudaSuccess;
+}
+
+// The status word, wait limit, device and context of a launch.
+cudaError_t dev_ctl(DevCtl* c) {
+  c->limit_ns = g_wait_limit_ns.load();
+  return status_ptr(&c->status, &c->dev, &c->ctx);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -118,21 +129,33 @@ bool encode_uncached(CUtensorMap* m, const MapKey& k) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Slot of a key: a hash of its fields picks one of two neighbouring slots
+// (the other one on a miss when the first is taken), so a lookup compares at
+// most two keys.
+size_t map_slot(const MapKey& k) {
+  uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+  for (int i = 0; i < 4; ++i) h = (h ^ k.d[i]) * 0x100000001B3ull;
+  h ^= static_cast<uint64_t>(k.kind) * 31 + static_cast<uint64_t>(k.box_rows);
+  return static_cast<size_t>((h >> 29) % (kMapSlots / 2)) * 2;
+}
+
 bool encode_cached(CUtensorMap* m, const MapKey& k) {
+  const size_t i = map_slot(k);
   std::lock_guard<std::mutex> lk(g_map_mu);
-  MapSlot* victim = &g_map_slots[0];
-  for (MapSlot& s : g_map_slots) {
+  for (size_t j = i; j < i + 2; ++j) {
+    MapSlot& s = g_map_slots[j];
     if (s.used && s.key == k) {
       s.used = ++g_map_clock;
       *m = s.map;
       return true;
     }
-    if (s.used < victim->used) victim = &s;
   }
   if (!encode_uncached(m, k)) return false;
-  victim->key = k;
-  victim->map = *m;
-  victim->used = ++g_map_clock;
+  // replace the less recently used of the two
+  MapSlot& v = g_map_slots[g_map_slots[i].used <= g_map_slots[i + 1].used ? i : i + 1];
+  v.key = k;
+  v.map = *m;
+  v.used = ++g_map_clock;
   return true;
 }
 
@@ -182,17 +205,16 @@ int fwd_lowbit_impl(int bits, const void* q_codes, const float* q_scales, const 
   if (bits == 4 && (!aligned32(q_codes) || !aligned32(k_codes))) return DIFFATTN_ERR_INVALID_ARG;
   if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const bool codes_ok = bits == 4 ? encode_4d_e2m1(&tq, q_codes, d, 2ull * H, N, B) &&
                                         encode_4d_e2m1(&tk, k_codes, d, 2ull * H, N, B)
                                   : encode_4d(&tq, q_codes, d, 2ull * H, N, B, 1) &&
                                         encode_4d(&tk, k_codes, d, 2ull * H, N, B, 1);
-  if (!codes_ok || !encode_4d(&tv, v, 2ull * d, H, N, B)) return DIFFATTN_ERR_CUDA;
+  if (!codes_ok || !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
+    return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
-  cudaError_t e = status_ptr(&ctl.status);
-  if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
-  ctl.limit_ns = g_wait_limit_ns.load();
-  return cuda_status(launch_prefill_sm100(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
+  if (dev_ctl(&ctl) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  return cuda_status(launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps,
                                           mode, q_scales, k_scales, bits, ctl, stream));
 }
 
@@ -347,16 +369,14 @@ int diffattn_fwd_mode(const void* q, const void* k, const void* v, void* o, int 
                                                causal, lambda, lambda_init, rms_w, eps, mode, stream));
   }
   if (d != 64 && d != 128) return DIFFATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
-      !encode_4d(&tv, v, 2ull * d, H, N, B))
+      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
-  cudaError_t e = status_ptr(&ctl.status);
-  if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
-  ctl.limit_ns = g_wait_limit_ns.load();
+  if (dev_ctl(&ctl) != cudaSuccess) return DIFFATTN_ERR_CUDA;
   return cuda_status(
-      launch_prefill_sm100(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, nullptr,
+      launch_prefill_sm100(tq, tk, tv, to, o, B, N, H, d, causal, lambda, lambda_init, rms_w, eps, mode, nullptr,
                            nullptr, 16, ctl, stream));
 }
 
@@ -443,15 +463,15 @@ int diffattn_fwd_train(const void* q, const void* k, const void* v, void* o, int
   if (B > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
   const BwdTcLayout L = bwd_tc_layout(B, N, H, d);
   if (!workspace || ws_bytes < L.bytes || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode_4d(&tq, q, d, 2ull * H, N, B) || !encode_4d(&tk, k, d, 2ull * H, N, B) ||
-      !encode_4d(&tv, v, 2ull * d, H, N, B))
+      !encode_4d(&tv, v, 2ull * d, H, N, B) || !encode_4d(&to, o, 2ull * d, H, N, B))
     return DIFFATTN_ERR_CUDA;
   DevCtl ctl;
   if (status_ptr(&ctl.status) != cudaSuccess) return DIFFATTN_ERR_CUDA;
   ctl.limit_ns = g_wait_limit_ns.load();
   char* ws = static_cast<char*>(workspace);
-  return cuda_status(launch_prefill_sm100_stats(tq, tk, tv, o, B, N, H, d, causal, lambda, lambda_init, rms_w,
+  return cuda_status(launch_prefill_sm100_stats(tq, tk, tv, &to, o, B, N, H, d, causal, lambda, lambda_init, rms_w,
                                                 eps, mode, reinterpret_cast<float*>(ws + L.off_omaps),
                                                 reinterpret_cast<float*>(ws + L.off_stats), L.n_pad, ctl, stream));
 }
@@ -538,6 +558,7 @@ int diffattn_decode_mode(const void* q, const void* k_cache, const void* v_cache
     return DIFFATTN_ERR_INVALID_ARG;
   if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   if (S > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (!decode_units_fit(S, H, max_seqlen)) return DIFFATTN_ERR_UNSUPPORTED;
   const size_t need = decode_workspace_bytes(S, H, d, max_seqlen);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return DIFFATTN_ERR_WORKSPACE;
   return cuda_status(launch_decode(q, k_cache, v_cache, cu_seqlens, max_seqlen, o, S, H, d, lambda, lambda_init,

@@ -557,7 +557,7 @@ cudaError_t launch_bwd_sm100_d(const BwdTcMaps& m, const void* dy, int B, int N,
   if (e == cudaSuccess) e = cudaMemsetAsync(dlambda, 0, sizeof(float), stream);
   if (e != cudaSuccess) return e;
   if (!stats_ready) {
-    e = launch_prefill_sm100_stats(m.q128, m.k128, m.v128, nullptr, B, N, H, D, causal, lambda, lambda_init,
+    e = launch_prefill_sm100_stats(m.q128, m.k128, m.v128, nullptr, nullptr, B, N, H, D, causal, lambda, lambda_init,
                                    rms_w, eps, mode, o_maps, reinterpret_cast<float*>(stats), L.n_pad, ctl, stream);
     if (e != cudaSuccess) return e;
   }

@@ -13,8 +13,10 @@
 //     each sequence (ceil(L / 512) chunks of up to 512 keys, at least one),
 //     so that the next kernel visits only chunks that exist.
 //   * decode_partial_kernel: a persistent grid (as many CTAs as fit on the
-//     GPU at once, spread over the heads) walks the chunks with a fixed
-//     stride.  Each warp streams its keys with 16-byte non-allocating loads,
+//     GPU at once) takes (chunk, head) units from a counter one at a time,
+//     so that every CTA keeps working until the units run out whatever the
+//     mix of full and partial chunks.  Each warp streams its keys with
+//     16-byte non-allocating loads,
 //     8 keys in flight per lane group; lane l holds elements [8l, 8l+8) of
 //     the 256-wide K row (lanes 0-15: map 1, lanes 16-31: map 2) and of the V
 //     row.  The 8 partial dot products are reduced across 16 lanes with a
@@ -25,7 +27,7 @@
 //     sequence's chunks with the log-sum-exp rescale per map, forms
 //     o1/l1 - lambda o2/l2, and applies the RMSNorm and scale.
 // Workspace: the chunk records (room for S * ceil(max_seqlen / 512) chunks
-// per head), then the S + 1 chunk offsets.
+// per head), then the S + 1 chunk offsets and the work counter.
 #include <math.h>
 
 #include "common.cuh"
@@ -66,6 +68,7 @@ __device__ __forceinline__ int seq_keys(const int* __restrict__ cu, int s, int S
 }
 
 // chunk_start[s] = chunks of the sequences before s; chunk_start[S] = all chunks.
+// chunk_start[S + 1] is the partial kernel's work counter: set to 0 here.
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int* __restrict__ cu_seqlens, int S,
                                                            int max_seqlen, int* __restrict__ chunk_start,
                                                            int* dbg) {
@@ -104,22 +107,36 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int* __restrict
     carry += warp_sum[31];
     __syncthreads();  // warp_sum is rewritten by the next pass
   }
-  if (threadIdx.x == 0) chunk_start[S] = carry;
+  if (threadIdx.x == 0) {
+    chunk_start[S] = carry;
+    chunk_start[S + 1] = 0;
+  }
 }
 
 __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
     const int* __restrict__ cu_seqlens, int S, int max_seqlen, int H, const int* __restrict__ chunk_start,
     float* __restrict__ ws, int* dbg) {
-  const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = lane >> 4;  // 0: map 1, 1: map 2
   const int hl = lane & 15;
   const int total = chunk_start[S];
+  int* next = const_cast<int*>(chunk_start) + S + 1;  // work counter: (chunk, head) units handed out
   __shared__ float sm_m[kWarps][2], sm_l[kWarps][2];
   __shared__ float sm_o[kWarps][2][kDV];
+  __shared__ int s_unit[2];  // this CTA's current and next unit
 
-  for (int c = blockIdx.x; c < total; c += gridDim.x) {
+  // Units are taken from the counter one at a time (the next one while the
+  // current is processed), so a CTA that drew short chunks takes more of
+  // them and all finish together.  Unit u is chunk u / H of head u % H.
+  const int units = total * H;
+  if (threadIdx.x == 0) s_unit[0] = atomicAdd(next, 1);
+  __syncthreads();
+  for (int it = 0;; ++it) {
+    const int u = s_unit[it & 1];
+    if (u >= units) break;
+    if (threadIdx.x == 0) s_unit[(it + 1) & 1] = atomicAdd(next, 1);
+    const int c = u / H, h = u % H;
     // the sequence of chunk c: the last s with chunk_start[s] <= c
     int s = 0;
     {
@@ -286,7 +303,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
         rec[2 * mp + 1] = Ls;
       }
     }
-    __syncthreads();  // the merge buffers are refilled by the next chunk
+    __syncthreads();  // the merge buffers are refilled by the next chunk; the next unit is visible
   }
 }
 
@@ -342,7 +359,7 @@ size_t plan_offset(int S, int H, int max_seqlen) {
 
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen) {
   if (S <= 0 || H <= 0 || d != kD || max_seqlen <= 0) return 0;
-  return plan_offset(S, H, max_seqlen) + ((static_cast<size_t>(S + 1) * sizeof(int) + 15) & ~static_cast<size_t>(15));
+  return plan_offset(S, H, max_seqlen) + ((static_cast<size_t>(S + 2) * sizeof(int) + 15) & ~static_cast<size_t>(15));
 }
 
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
@@ -350,8 +367,8 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
                           const float* rms_w, float eps, int mode, void* workspace, cudaStream_t stream) {
   (void)d;
   int* dbg = debug_status();
-  // persistent partial grid: the CTAs that fit on the GPU at once, spread over
-  // the heads (looked up once per device)
+  // persistent partial grid: the CTAs that fit on the GPU at once (looked up
+  // once per device)
   static int resident[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -367,16 +384,15 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
   }
   const long long max_chunks = (static_cast<long long>(max_seqlen) + kChunk - 1) / kChunk;
   const long long upper = static_cast<long long>(S) * max_chunks;  // chunks there can be
-  long long gx = resident[dev] / H;
+  long long gx = resident[dev];
+  if (gx > upper * H) gx = upper * H;
   if (gx < 1) gx = 1;
-  if (gx > upper) gx = upper;
-  if (gx > 0x7fffffffll) gx = 0x7fffffffll;
   float* recs = static_cast<float*>(workspace);
   int* chunk_start = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan_offset(S, H, max_seqlen));
   decode_plan_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, S, max_seqlen, chunk_start, dbg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_partial_kernel<<<dim3(static_cast<unsigned>(gx), H), kWarps * 32, 0, stream>>>(
+  decode_partial_kernel<<<static_cast<unsigned>(gx), kWarps * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
       static_cast<const __nv_bfloat16*>(v_cache), cu_seqlens, S, max_seqlen, H, chunk_start, recs, dbg);
   e = cudaGetLastError();

@@ -77,6 +77,7 @@ extern "C" int diffattn_decode_noalloc(const void* q, const void* k_cache, const
     return DIFFATTN_ERR_INVALID_ARG;
   if (d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   if (S > 65535 || H > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (!diffattn::decode_units_fit(S, H, max_seqlen)) return DIFFATTN_ERR_UNSUPPORTED;
   const size_t need = diffattn::decode_workspace_bytes(S, H, d, max_seqlen);
   if (need == 0 || need > kScratchBytes) return DIFFATTN_ERR_WORKSPACE;  // beyond the built-in scratch
   void* scratch = nullptr;

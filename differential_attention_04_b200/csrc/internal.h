@@ -31,6 +31,8 @@ inline int* debug_status() {
 struct DevCtl {
   int* status;
   unsigned long long limit_ns;
+  int dev = -1;                  // the current device, when the caller looked it up
+  unsigned long long ctx = 0;    // its context's id (current_context_id), when looked up
 };
 
 cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
@@ -48,10 +50,11 @@ __host__ __device__ inline float map2_coefficient(int mode, float lam) {
 
 // Tensor-core (tcgen05) prefill, d in {64, 128} for bf16 queries and keys,
 // d = 128 for low-bit ones (q_scale, k_scale non-null; qk_bits 8: e4m3 codes,
-// 4: packed e2m1 codes).  tq/tk map [B, N, H*2, d]; tv maps [B, N, H, 2d];
-// boxes are 128 bytes (bf16, e4m3) or 128 elements (e2m1) x 128 rows with
-// 128-byte swizzle.  The output o [B, N, H, 2d] (bf16) is written directly.
-cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+// 4: packed e2m1 codes).  tq/tk map [B, N, H*2, d]; tv and to map
+// [B, N, H, 2d]; boxes are 128 bytes (bf16, e4m3) or 128 elements (e2m1) x
+// 128 rows with 128-byte swizzle.
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, int mode, const float* q_scale,
                                  const float* k_scale, int qk_bits, DevCtl ctl, cudaStream_t stream);
@@ -92,9 +95,9 @@ cudaError_t launch_bwd_sm100(const BwdTcMaps& m, const void* dy, int B, int N, i
                              bool stats_ready, DevCtl ctl, cudaStream_t stream);
 // The tcgen05 prefill in its statistics mode: per map, O_i / l_i into
 // o_maps and the log2-sum-exp into component i of the float4 rows of lse;
-// with o non-null, the normalised output too.
+// with `to` (the output map over o) non-null, the normalised output too.
 cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                       void* o, int B, int N, int H, int d, int causal,
+                                       const CUtensorMap* to, void* o, int B, int N, int H, int d, int causal,
                                        const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                                        float* o_maps, float* lse, int n_pad, DevCtl ctl, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int d,
@@ -123,6 +126,12 @@ cudaError_t launch_rope_table(int seq_len, int d, double base, float* table, cud
 
 // Split-KV decode (bf16, d = 128).
 size_t decode_workspace_bytes(int S, int H, int d, int max_seqlen);
+// Whether S * ceil(max_seqlen / 512) * H (chunk, head) units stay within the
+// kernels' 32-bit counters.
+inline bool decode_units_fit(int S, int H, int max_seqlen) {
+  const long long chunks = (static_cast<long long>(max_seqlen) + 511) / 512;
+  return static_cast<long long>(S) * chunks * H <= 0x3fffffffll;
+}
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int* cu_seqlens,
                           int max_seqlen, void* o, int S, int H, int d, const float* lambda, float lambda_init,
                           const float* rms_w, float eps, int mode, void* workspace, cudaStream_t stream);

@@ -13,51 +13,50 @@
 //   (batch, head).  The (batch, head) pairs are taken in groups whose K and V
 //   fit in about 48 MB of L2 together; within a group the items are ordered
 //   longest first (causal: the last query tiles); the whole list is dealt to
-//   the clusters in a snake.  Per item, CTA rank i computes map i+1 only:
-//   S_i = Q_i K_i^T on the tensor cores, its own online softmax (running max
-//   m_i and sum l_i per row), and O_i += P_i V.  Both CTAs stream the same V
-//   tiles.  Tensor memory per CTA (512 columns): S (fp32, one buffer) in
-//   columns [0, 128), P (bf16, two buffers of 64 columns) in [128, 256), O_i
-//   in [256, 256 + 2d).  P feeds the PV product straight from tensor memory.
+//   the clusters in a snake.  Per item, CTA rank i
+//   computes map i+1 only: S_i = Q_i K_i^T on the tensor cores,
+//   its own online softmax (running max m_i and sum l_i per row), and
+//   O_i += P_i V.  Both CTAs stream the same V tiles.  Tensor memory per CTA
+//   (512 columns): S (fp32, one buffer) in columns [0, 128), P (bf16, two
+//   buffers of 64 columns) in [128, 256), O_i in [256, 256 + 2d).  P feeds
+//   the PV product straight from tensor memory.  Keeping P apart from S lets
+//   S_{j+1} be computed as soon as the softmax has read S_j into registers.
+//   The epilogue exchanges half of the columns through distributed shared
+//   memory: rank 0 keeps output columns [0, d), rank 1 keeps [d, 2d); each
+//   bulk-copies the other half of its O_i/l_i (scaled by -lambda on rank 1)
+//   into the partner's shared memory, the partial sums of squares of each
+//   row are swapped, and each CTA stages its columns of
+//   (1 - lambda_init) * w * O / rms as bf16 and writes them with TMA stores.
+//   The two CTAs meet through mbarriers only (each side says when its
+//   receive buffer is free, the copies complete on the receiver's barrier,
+//   and so do the sums of squares, sent with st.async), so the producer and
+//   MMA threads run on into the next item: its Q and K tiles load and its
+//   first S product runs while the epilogue finishes.  Warp 3 stores each
+//   output tile, so the softmax warps start the next item as soon as the tile
+//   is staged.
 //
-// The epilogue runs beside the next item
-//   A warpgroup of its own drains each finished O_i out of tensor memory, so
-//   the softmax warps go straight on to the next item and the tensor cores
-//   only wait for the drain (two TMEM reads per row) before the next item's
-//   first PV.  Rank 0 keeps output columns [0, d), rank 1 keeps [d, 2d): each
-//   sends the other half of its O_i / l_i (scaled by c = -lambda on rank 1)
-//   straight from registers into the partner's shared memory with st.async,
-//   holds its own half in registers, adds the partner's half when it lands,
-//   swaps the partial sums of squares of each row, and stores
-//   (1 - lambda_init) * w * O / rms as bf16 straight to global memory.  The
-//   receive buffer is the V stage of the item's last tile; the V producer
-//   reloads that stage only once the epilogue has released it.  The two CTAs
-//   meet through mbarriers only.
-//
-// Warp roles (384 threads; registers re-split per warpgroup at start-up)
+// Warp roles (256 threads)
 //   warp 0: TMA producer for Q_i and K_i      warp 2: TMA producer for V
 //   warp 1: tensor-memory allocator + the single MMA-issuing thread
-//   warp 3: idle
-//   warps 4-7: softmax, one query row per thread
-//   warps 8-11: epilogue, one query row per thread
+//   warp 3: TMA store of each output tile     warps 4-7: softmax + epilogue,
+//                                             one query row per thread
 //
-// Pipeline per key tile j (P buffer and K/V stage b = j % 2), one stream of
-// tiles across all items.  A tcgen05.mma issue returns only when the
-// instruction is nearly done, so the issue order decides what overlaps:
-//   MMA:     wait s_free (the softmax has read the previous S) -> S_j ->
-//            commit s_full, k_empty; then wait p_full of the previous tile
-//            (the last tile of the previous item at an item's first tile) ->
-//            O += P V -> commit v_empty, p_empty.  The first PV of an item also
-//            waits until the epilogue has drained the previous item's O.
+// Pipeline per key tile j (P buffer and K/V stage b = j % 2).  A
+// tcgen05.mma issue returns only when the instruction is nearly done, so the
+// issue order decides what overlaps:
+//   MMA:     wait s_free (the softmax has read S_{j-1}) -> S_j -> commit
+//            s_full, k_empty; then wait p_full[b'] of tile j-1 ->
+//            O += P_{j-1} V_{j-1} -> commit v_empty, p_empty[b'].  PV_{j-1}
+//            thus runs while the softmax works on tile j, and S_{j+1} is
+//            ready when the softmax finishes it.
 //   softmax: wait s_full (S_j done, and so every MMA issued before it:
-//            PV_{j-2} included, the last reader of P[b]); read the 128 scores of
-//            its row; arrive s_free; mask; P = exp2(s*c - m) as bf16 into P[b],
-//            relative to the reference maximum m, while forming the tile's own
-//            maximum; arrive p_full[b].  Lazy rescale: only when the running
-//            maximum exceeds m by more than 2^8 are O and l rescaled to it, once
-//            PV_j has completed; a jump beyond 2^64, which could overflow P,
-//            rescales first and recomputes P.  At the end of an item the row's
-//            l (and log-sum-exp) go to shared memory for the epilogue.
+//            PV_{j-2}, the last reader of P[b]); read the 128 scores of its
+//            row; arrive s_free; mask; P = exp2(s*c - m) as bf16 into P[b],
+//            relative to the reference maximum m, while forming the tile's
+//            own maximum; arrive p_full[b].  Lazy rescale: only when the
+//            running maximum exceeds m by more than 2^8 are O and l rescaled
+//            to it, once PV_j has completed; a jump beyond 2^64, which could
+//            overflow P, rescales first and recomputes P.
 #include <math.h>
 
 #include "common.cuh"
@@ -67,19 +66,12 @@ namespace diffattn {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 256;
 constexpr int kBM = 128;  // query rows per CTA
 constexpr int kBN = 128;  // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kOverflowGuard = 64.0f;    // log2 units
-// Registers per thread of each warpgroup after start-up (the block launches
-// with 168 each: 384 x 168 = 64512, which the three shares use up; this
-// split leaves the bf16, e4m3 and e2m1 forward kernels without spills).
-constexpr uint32_t kRegsProducer = 80;  // warps 0-3: TMA producers, MMA issuer
-constexpr uint32_t kRegsSoftmax = 248;  // warps 4-7
-constexpr uint32_t kRegsEpilogue = 176; // warps 8-11
-static_assert(128 * (kRegsProducer + kRegsSoftmax + kRegsEpilogue) <= kThreads * 168, "register split");
 
 // QK8: queries and keys arrive as low-bit codes with a float32 scale per
 // (batch, head, map) and S is a kind::f8f6f4 product: e4m3 codes take one
@@ -105,16 +97,17 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + 2 * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + 2 * V_BYTES;
   static constexpr int OFF_SSX = OFF_BAR + 256;  // float[128]: the partner's sums of squares
-  static constexpr int OFF_LM = OFF_SSX + 512;   // float2[128]: each row's (l, log-sum-exp) for the epilogue
-  static constexpr int SMEM_USED = OFF_LM + 1024;
+  static constexpr int SMEM_USED = OFF_SSX + 512;
   static constexpr int EXCH_BYTES = kBM * HALF * 4;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
   static constexpr uint32_t TM_S = 0;            // S (fp32, 128 columns)
   static constexpr uint32_t TM_P = 128;          // P buffer b (bf16 pairs) at column TM_P + 64 * b
   static constexpr uint32_t TM_O = 256;
   static constexpr uint32_t TM_COLS = 512;
-  static_assert(EXCH_BYTES <= V_BYTES, "the receive buffer must fit in one V stage");
+  static_assert(EXCH_BYTES <= V_BYTES, "exchange buffers must fit in one V stage each");
+  static_assert(kBM * HALF * 2 <= V_BYTES, "output staging must fit in one V stage");
   static_assert(SMEM_USED + 1024 <= 232448, "shared memory per CTA");
+
 };
 
 struct Bars {
@@ -124,16 +117,13 @@ struct Bars {
   uint64_t s_full, s_free;
   uint64_t p_full[2], p_empty[2];
   uint64_t mma_done;
-  uint64_t sm_done[2];    // item k (slot k % 2): the softmax has finished its rows (l, any rescale of O)
-  uint64_t o_free;        // per item: the epilogue has drained O (and read l)
-  uint64_t exch_full;     // per item: the partner's half of the output has landed here
-  uint64_t peer_ready;    // per item: the partner's receive buffer is armed and free (remote arrive)
-  uint64_t ss_full;       // per item: the partner's sums of squares are here
-  uint64_t epi_free[2];   // item k (slot k % 2): the epilogue has released its receive buffer
+  uint64_t exch_full;   // per item: the partner's half of the output has landed here
+  uint64_t peer_ready;  // per item: the partner's receive buffer is free (remote arrive)
+  uint64_t ss_full;     // per item: the partner's sums of squares are here (remote arrive)
+  uint64_t epi_free;    // per item: the epilogue is done with the V stages
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars) <= 256, "barrier area");
 
 }  // namespace
 
@@ -176,7 +166,8 @@ enum : int { kQkBf16 = 0, kQkE4m3 = 1, kQkE2m1 = 2 };
 template <int D, int QKF, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                         const __grid_constant__ CUtensorMap tv, const PrefillParams p) {
+                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                         const PrefillParams p) {
   constexpr bool QK8 = QKF != kQkBf16;
   using C = Cfg<D, QK8>;
   // bytes a Q / K tile brings in from global memory (packed e2m1: half its shared-memory size)
@@ -189,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + C::OFF_V;
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   float* ssx = reinterpret_cast<float*>(smem + C::OFF_SSX);
-  float2* lm = reinterpret_cast<float2*>(smem + C::OFF_LM);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();  // 0: map 1, 1: map 2
@@ -231,16 +221,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_empty[i], 1);
       mbar_init(&bars->p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&bars->p_empty[i], 1);
-      mbar_init(&bars->sm_done[i], 4);  // one arrival per softmax warp
-      mbar_init(&bars->epi_free[i], 1);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 4);
     mbar_init(&bars->mma_done, 1);
-    mbar_init(&bars->o_free, 1);
     mbar_init(&bars->exch_full, 1);
     mbar_init(&bars->peer_ready, 1);
     mbar_init(&bars->ss_full, 1);
+    mbar_init(&bars->epi_free, 1);
     bars->abort = 0;
     fence_mbarrier_init();
   }
@@ -248,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&to);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, C::TM_COLS);
@@ -264,174 +253,180 @@ __global__ void __launch_bounds__(kThreads, 1)
   int drain_abort = 0;
   const WaitCtl wdrain{p.status, &drain_abort, 1000000000ull};
 
-  if (warp < 4) {
-    regs_dec<kRegsProducer>();
-    if (warp == 0) {
-      // -------------------------------------------------- Q / K producer --
-      if (lane == 0) {
-        int gk = 0;  // K tiles issued (all items)
-        bool ok = true;
-        for (int k = 0; ok; ++k) {
-          const int idx = item_of(k);
-          if (idx < 0) break;
-          const Item it = decode(idx);
-          const int c1 = 2 * it.h + static_cast<int>(rank);
-          // Q of this item replaces the last one's once that item's S products have read it
-          if (k > 0 && !(ok = mbar_wait(&bars->q_empty, (k - 1) & 1, wc))) break;
-          // debug builds: the tile lies in the tensor (else the load is skipped
-          // and the phase completed without data)
-          if (DA_CHECK(p.status, it.b >= 0 && it.b < p.B && it.h >= 0 && c1 < 2 * p.H && it.qtile >= 0 &&
-                                     it.qtile * kBM < N)) {
-            mbar_arrive_expect_tx(&bars->q_full, kQTx);
+  if (warp == 0) {
+    // ---------------------------------------------------- Q / K producer --
+    if (lane == 0) {
+      int gk = 0;  // K tiles issued (all items)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        const int c1 = 2 * it.h + static_cast<int>(rank);
+        // Q of this item replaces the last one's once that item's S products have read it
+        if (k > 0 && !(ok = mbar_wait(&bars->q_empty, (k - 1) & 1, wc))) break;
+        // debug builds: the tile lies in the tensor (else the load is skipped
+        // and the phase completed without data)
+        if (DA_CHECK(p.status, it.b >= 0 && it.b < p.B && it.h >= 0 && c1 < 2 * p.H && it.qtile >= 0 &&
+                                   it.qtile * kBM < N)) {
+          mbar_arrive_expect_tx(&bars->q_full, kQTx);
+#pragma unroll
+          for (int blk = 0; blk < C::QBLK; ++blk)
+            tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * C::QBOX, c1, it.qtile * kBM, it.b);
+        } else {
+          mbar_arrive(&bars->q_full);
+        }
+        for (int j = 0; j < it.n_kv; ++j, ++gk) {
+          const int st = gk & 1;
+          if (!(ok = mbar_wait(&bars->k_empty[st], ((gk >> 1) & 1) ^ 1, wc))) break;
+          if (DA_CHECK(p.status, j * kBN < N)) {
+            mbar_arrive_expect_tx(&bars->k_full[st], kKTx);
 #pragma unroll
             for (int blk = 0; blk < C::QBLK; ++blk)
-              tma_load_4d(sQ + blk * C::BLK_BYTES, &tq, &bars->q_full, blk * C::QBOX, c1, it.qtile * kBM, it.b);
+              tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * C::QBOX, c1,
+                          j * kBN, it.b);
           } else {
-            mbar_arrive(&bars->q_full);
-          }
-          // The next item's Q can only load once this item's last S product
-          // has read the buffer; start it on its way to L2 now, so that the
-          // load at the item boundary is an L2 hit.
-          {
-            const int nidx = item_of(k + 1);
-            if (nidx >= 0) {
-              const Item nt = decode(nidx);
-#pragma unroll
-              for (int blk = 0; blk < C::QBLK; ++blk)
-                tma_prefetch_l2_4d(&tq, blk * C::QBOX, 2 * nt.h + static_cast<int>(rank), nt.qtile * kBM, nt.b);
-            }
-          }
-          for (int j = 0; j < it.n_kv; ++j, ++gk) {
-            const int st = gk & 1;
-            if (!(ok = mbar_wait(&bars->k_empty[st], ((gk >> 1) & 1) ^ 1, wc))) break;
-            if (DA_CHECK(p.status, j * kBN < N)) {
-              mbar_arrive_expect_tx(&bars->k_full[st], kKTx);
-#pragma unroll
-              for (int blk = 0; blk < C::QBLK; ++blk)
-                tma_load_4d(sK + st * C::K_BYTES + blk * C::BLK_BYTES, &tk, &bars->k_full[st], blk * C::QBOX, c1,
-                            j * kBN, it.b);
-            } else {
-              mbar_arrive(&bars->k_full[st]);
-            }
+            mbar_arrive(&bars->k_full[st]);
           }
         }
-        // nothing may still be landing in shared memory when the CTA exits
-        for (int j = max(0, gk - 2); j < gk; ++j) mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, wdrain);
       }
-      __syncwarp();
-    } else if (warp == 2) {
-      // ------------------------------------------------------ V producer --
-      if (lane == 0) {
-        int gv = 0;  // V tiles issued (all items)
-        // last tiles (global indices) of the two previous items: the epilogue
-        // of an item holds the V stage of its last tile as its receive buffer
-        int last1 = -8, last2 = -8;  // items k-1 and k-2 (none yet: below any gv - 2)
-        bool ok = true;
-        for (int k = 0; ok; ++k) {
-          const int idx = item_of(k);
-          if (idx < 0) break;
-          const Item it = decode(idx);
-          for (int j = 0; j < it.n_kv; ++j, ++gv) {
-            const int st = gv & 1;
-            // the stage's previous tile, gv - 2, may have been an item's last:
-            // its epilogue must have released the stage first
-            if (gv - 2 == last1 && !(ok = mbar_wait(&bars->epi_free[(k - 1) & 1], ((k - 1) >> 1) & 1, wc))) break;
-            if (gv - 2 == last2 && !(ok = mbar_wait(&bars->epi_free[(k - 2) & 1], ((k - 2) >> 1) & 1, wc))) break;
-            if (!(ok = mbar_wait(&bars->v_empty[st], ((gv >> 1) & 1) ^ 1, wc))) break;
-            if (DA_CHECK(p.status, it.b >= 0 && it.b < p.B && it.h >= 0 && it.h < p.H && j * kBN < N)) {
-              mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
+      // nothing may still be landing in shared memory when the CTA exits
+      for (int j = max(0, gk - 2); j < gk; ++j) mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, wdrain);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // -------------------------------------------------------- V producer --
+    if (lane == 0) {
+      int gv = 0;  // V tiles issued (all items)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        // the previous item's epilogue uses both V stages for its exchange
+        if (k > 0 && !(ok = mbar_wait(&bars->epi_free, (k - 1) & 1, wc))) break;
+        for (int j = 0; j < it.n_kv; ++j, ++gv) {
+          const int st = gv & 1;
+          if (!(ok = mbar_wait(&bars->v_empty[st], ((gv >> 1) & 1) ^ 1, wc))) break;
+          if (DA_CHECK(p.status, it.b >= 0 && it.b < p.B && it.h >= 0 && it.h < p.H && j * kBN < N)) {
+            mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
 #pragma unroll
-              for (int blk = 0; blk < C::VBLK; ++blk)
-                tma_load_4d(sV + st * C::V_BYTES + blk * C::BLK_BYTES, &tv, &bars->v_full[st], blk * 64, it.h,
-                            j * kBN, it.b);
-            } else {
-              mbar_arrive(&bars->v_full[st]);
-            }
+            for (int blk = 0; blk < C::VBLK; ++blk)
+              tma_load_4d(sV + st * C::V_BYTES + blk * C::BLK_BYTES, &tv, &bars->v_full[st], blk * 64, it.h,
+                          j * kBN, it.b);
+          } else {
+            mbar_arrive(&bars->v_full[st]);
           }
-          last2 = last1;
-          last1 = gv - 1;
         }
-        for (int j = max(0, gv - 2); j < gv; ++j) mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, wdrain);
       }
-      __syncwarp();
-    } else if (warp == 1) {
-      // ----------------------------------------------------- MMA issuer --
-      if (lane == 0) {
-        constexpr uint32_t idesc_s = QKF == kQkE2m1   ? idesc_f8f6f4_f32(128, 128, kF8f6f4E2m1)
-                                     : QKF == kQkE4m3 ? idesc_f8f6f4_f32(128, 128, kF8f6f4E4m3)
-                                                      : idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
-        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-        // O (+)= P V for global tile g (P buffer and V stage g % 2); `first`
-        // starts item `k`'s O, which waits until the epilogue has drained item k-1's
-        auto issue_pv = [&](int g, bool first, int k) -> bool {
-          const int bb = g & 1;
-          const uint32_t ph = (g >> 1) & 1;
-          if (!mbar_wait(&bars->v_full[bb], ph, wc)) return false;
-          if (!mbar_wait(&bars->p_full[bb], ph, wc)) return false;
-          if (first && k > 0 && !mbar_wait(&bars->o_free, (k - 1) & 1, wc)) return false;
+      for (int j = max(0, gv - 2); j < gv; ++j) mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, wdrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = QKF == kQkE2m1   ? idesc_f8f6f4_f32(128, 128, kF8f6f4E2m1)
+                                   : QKF == kQkE4m3 ? idesc_f8f6f4_f32(128, 128, kF8f6f4E4m3)
+                                                    : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      int gs = 0;  // S products issued (all items)
+      int gp = 0;  // PV products issued (all items)
+      // O (+)= P V for the next tile, with P from buffer gp % 2 and V from stage gp % 2;
+      // `first` starts a new item's O
+      auto issue_pv = [&](bool first) -> bool {
+        const int bb = gp & 1;
+        const uint32_t ph = (gp >> 1) & 1;
+        if (!mbar_wait(&bars->v_full[bb], ph, wc)) return false;
+        if (!mbar_wait(&bars->p_full[bb], ph, wc)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t a_tmem = tmem + C::TM_P + 64 * bb + 8 * kk;
+          const uint64_t bd = smem_desc_sw128(sVa + bb * C::V_BYTES + kk * 2048, C::BLK_BYTES, 1024);
+          umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->v_empty[bb]);
+        umma_commit(&bars->p_empty[bb]);
+        ++gp;
+        return true;
+      };
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        if (!(ok = mbar_wait(&bars->q_full, k & 1, wc))) break;
+        for (int j = 0; ok && j < it.n_kv; ++j, ++gs) {
+          const int st = gs & 1;
+          // S overwrites the previous S tile: every softmax warp must have read it
+          if (gs > 0 && !(ok = mbar_wait(&bars->s_free, (gs - 1) & 1, wc))) break;
+          if (!(ok = mbar_wait(&bars->k_full[st], (gs >> 1) & 1, wc))) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint32_t a_tmem = tmem + C::TM_P + 64 * bb + 8 * kk;
-            const uint64_t bd = smem_desc_sw128(sVa + bb * C::V_BYTES + kk * 2048, C::BLK_BYTES, 1024);
-            umma_ts(tmem + C::TM_O, a_tmem, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < D / C::KSTEP; ++kk) {  // each instruction takes 32 bytes of every row
+            const int blk = kk >> 2;
+            const uint32_t koff = (kk & 3) * 32;
+            const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + koff, 16, 1024);
+            if constexpr (QK8)
+              umma_ss_f8(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            else
+              umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&bars->v_empty[bb]);
-          umma_commit(&bars->p_empty[bb]);
-          return true;
-        };
-        // One stream of tiles across all items: S of tile g, then PV of tile
-        // g - 1 (which may belong to the previous item).
-        bool ok = true;
-        int gs = 0;                  // S products issued (all items)
-        int pv_k = -1, pv_j = 0;     // item and tile-in-item of the pending PV (gs - 1)
-        for (int k = 0; ok; ++k) {
-          const int idx = item_of(k);
-          if (idx < 0) break;
-          const Item it = decode(idx);
-          if (!(ok = mbar_wait(&bars->q_full, k & 1, wc))) break;
-          for (int j = 0; j < it.n_kv; ++j, ++gs) {
-            const int st = gs & 1;
-            // S overwrites the previous S tile: every softmax warp must have read it
-            if (gs > 0 && !(ok = mbar_wait(&bars->s_free, (gs - 1) & 1, wc))) break;
-            if (!(ok = mbar_wait(&bars->k_full[st], (gs >> 1) & 1, wc))) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < D / C::KSTEP; ++kk) {  // each instruction takes 32 bytes of every row
-              const int blk = kk >> 2;
-              const uint32_t koff = (kk & 3) * 32;
-              const uint64_t ad = smem_desc_sw128(sQa + blk * C::BLK_BYTES + koff, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(sKa + st * C::K_BYTES + blk * C::BLK_BYTES + koff, 16, 1024);
-              if constexpr (QK8)
-                umma_ss_f8(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-              else
-                umma_ss(tmem + C::TM_S, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&bars->k_empty[st]);
-            umma_commit(&bars->s_full);
-            if (j == it.n_kv - 1) umma_commit(&bars->q_empty);  // the item's S products are all issued
-            if (gs > 0 && !(ok = issue_pv(gs - 1, pv_j == 0, pv_k))) break;
-            pv_k = k;
-            pv_j = j;
-          }
+          umma_commit(&bars->k_empty[st]);
+          umma_commit(&bars->s_full);
+          if (j == it.n_kv - 1) umma_commit(&bars->q_empty);  // the item's S products are all issued
+          if (j > 0) ok = issue_pv(j == 1);
         }
-        if (ok && gs > 0) issue_pv(gs - 1, pv_j == 0, pv_k);
-        // drain: every issued MMA has completed before tensor memory is freed
-        umma_commit(&bars->mma_done);
-        mbar_wait(&bars->mma_done, 0, wdrain);
+        if (ok) ok = issue_pv(it.n_kv == 1);
       }
-      __syncwarp();
+      // drain: every issued MMA has completed before tensor memory is read or freed
+      umma_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0, wdrain);
     }
-  } else if (warp < 8) {
-    // ---------------------------------------------------------- softmax --
-    regs_inc<kRegsSoftmax>();
+    __syncwarp();
+  } else if (warp == 3) {
+    // --------------------------------------------------- output store --
+    // Per item: once the softmax warps have staged the bf16 tile (V stage 1),
+    // store it with TMA, wait until the store has read it, and free both V
+    // stages for the next item.  The softmax warps do not wait for any of it.
+    if constexpr (OUT != kOutStats) {
+      const uint8_t* out_tile = sV + C::V_BYTES;
+      const int own0 = (rank == 0) ? 0 : C::HALF;
+      for (int k = 0;; ++k) {
+        const int idx = item_of(k);
+        if (idx < 0) break;
+        const Item it = decode(idx);
+        named_bar_sync(2, 160);  // with the softmax warps' arrivals
+        if (lane == 0) {
+#pragma unroll
+          for (int blk = 0; blk < C::HALF / 64; ++blk)  // rows >= N are clipped by the store
+            tma_store_4d(&to, out_tile + blk * C::BLK_BYTES, own0 + 64 * blk, it.h, it.qtile * kBM, it.b);
+          bulk_commit_group();
+          bulk_wait_group_read0();  // the stage must stay valid until the store has read it
+          mbar_arrive(&bars->epi_free);
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  if (warp >= 4) {
+    // ------------------------------------------------ softmax + epilogue --
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row within the tile (= TMEM lane)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float coef2 = map2_coefficient(p.mode, *p.lambda);  // c in softmax(S1) + c softmax(S2)
+    constexpr int HALF = C::HALF;
+    constexpr int NC = HALF / 4;  // float4 chunks per exchanged row
+    float* recv = reinterpret_cast<float*>(sV);              // V stage 0: the partner's half
+    float* stage = reinterpret_cast<float*>(sV + C::V_BYTES);  // V stage 1: the half sent, then the output
+    const uint32_t own0 = (rank == 0) ? 0 : HALF;   // columns this CTA finishes
+    const uint32_t send0 = (rank == 0) ? HALF : 0;  // columns it hands to the partner
     int g = 0;  // S / P tiles consumed (all items)
     bool sm_ok = true;
-    for (int k = 0; sm_ok; ++k) {
+    for (int k = 0;; ++k) {
       const int idx = item_of(k);
       if (idx < 0) break;
       const Item it = decode(idx);
@@ -457,9 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         l_run *= alpha;
       };
-      for (int j = 0; j < N_kv; ++j, ++g) {
+      for (int j = 0; sm_ok && j < N_kv; ++j, ++g) {
         const int bb = g & 1;
-        // every exit below is taken by the whole warp (a wait may end differently in its lanes)
+        // every exit is taken by the whole warp (a wait may end differently in its lanes)
         if (!(sm_ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, g & 1, wc)))) break;
         // S_g has completed, and with it every MMA issued before it, PV_{g-2}
         // included: P buffer b is free.
@@ -529,8 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         make_p(true);
         // A jump of the maximum by more than 2^64 would overflow P: rescale O
-        // to the new maximum (after the previous tile's PV has completed) and
-        // redo P.  Never on an item's first tile (it set the reference).
+        // to the new maximum (after the previous tile's PV has completed) and redo P.
         const bool hard = t_mx > m_run + kOverflowGuard;
         if (__any_sync(0xffffffffu, hard)) {
           tmem_st_wait();
@@ -556,53 +550,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (need) m_run = t_mx;
         }
       }
-      if (!sm_ok) break;
-      // Hand the row's l (and m + log2 l) to the epilogue once it has read the
-      // previous item's (it has when it drained that item's O).
-      if (k > 0 && !(sm_ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_free, (k - 1) & 1, wc)))) break;
-      lm[r] = make_float2(l_run, m_run + log2f(l_run));
-      tc_fence_before();  // any rescale of O (completed above) precedes the arrival
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sm_done[k & 1]);
-    }
-  } else {
-    // --------------------------------------------------------- epilogue --
-    regs_inc<kRegsEpilogue>();
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // query row within the tile (= TMEM lane)
-    const int etid = tid - 256;         // 0..127
-    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const float coef2 = map2_coefficient(p.mode, *p.lambda);  // c in softmax(S1) + c softmax(S2)
-    constexpr int HALF = C::HALF;
-    constexpr int NC = HALF / 4;  // float4 chunks per exchanged row
-    const uint32_t own0 = (rank == 0) ? 0 : HALF;   // columns this CTA finishes
-    const uint32_t send0 = (rank == 0) ? HALF : 0;  // columns it hands to the partner
-    const uint32_t peer_exch = map_to_cta(smem_u32(&bars->exch_full), partner);
-    const uint32_t peer_ss = map_to_cta(smem_u32(&bars->ss_full), partner);
-    const uint32_t peer_ssx = map_to_cta(smem_u32(ssx + r), partner);
-    int g_end = 0;  // tiles through the current item (all items)
-    bool ok = true;
-    for (int k = 0;; ++k) {  // leaves only through the group-wide decision below
-      const int idx = item_of(k);
-      if (idx < 0) break;
-      const Item it = decode(idx);
-      g_end += it.n_kv;
-      const int glast = g_end - 1;
-      const int qrow = it.qtile * kBM + r;
-      // the softmax has finished the item's rows, and its last PV (with every
-      // earlier MMA) has completed: O is final.  The decision to go on is taken
-      // by all 128 threads together (a wait may end differently in each), so
-      // every named barrier below is reached by all of them.
-      bool w_ok = ok && mbar_wait(&bars->sm_done[k & 1], (k >> 1) & 1, wc);
-      w_ok = w_ok && mbar_wait(&bars->p_empty[glast & 1], (glast >> 1) & 1, wc);
-      if (!(ok = named_bar_and(2, 128, w_ok))) break;
+      // the loop above may stop early after an abort: keep the tile count in step
+      g = 0;
+      for (int kk = 0; kk <= k; ++kk) g += decode(item_of(kk)).n_kv;
+
+      // ------------------------------------------------------ epilogue --
+      // O is complete once the item's last PV (and with it every earlier MMA) has.
+      if (sm_ok) sm_ok = mbar_wait(&bars->p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, wc);
       tc_fence_after();
-      const float2 lr = lm[r];
       if constexpr (OUT != kOutNorm) {
         // This map's O_i / l_i for the row, and lse_i = m + log2(l) in the
         // scaled log2 units of P = exp2(s * sc - m): P / l = exp2(s * sc - lse_i).
         const bool live = qrow < N && DA_CHECK(p.status, qrow < p.n_pad && it.b < p.B && it.h < p.H);
-        const float inv = 1.0f / lr.x;
+        const float inv = 1.0f / l_run;
         float* orow = p.o_maps + ((static_cast<size_t>(it.b) * N + (live ? qrow : 0)) * p.H + it.h) * (2 * C::DV) +
                       rank * C::DV;
 #pragma unroll 1
@@ -617,102 +577,97 @@ __global__ void __launch_bounds__(kThreads, 1)
                               __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
           }
         }
-        if (live) p.lse[((static_cast<size_t>(it.b) * p.H + it.h) * p.n_pad + qrow) * 4 + rank] = lr.y;
+        if (live) p.lse[((static_cast<size_t>(it.b) * p.H + it.h) * p.n_pad + qrow) * 4 + rank] = m_run + log2f(l_run);
         if constexpr (OUT == kOutStats) {
           tc_fence_before();
-          named_bar_sync(2, 128);  // every row's tensor-memory reads are done
-          if (etid == 0) {
-            mbar_arrive(&bars->o_free);            // the next item's first PV may overwrite O
-            mbar_arrive(&bars->epi_free[k & 1]);   // no receive buffer held
-          }
+          named_bar_sync(1, 128);  // every row's tensor-memory reads are done
+          if (tid == 128) mbar_arrive(&bars->epi_free);  // the next item's first PV may overwrite O
           __syncwarp();
           continue;
         }
+        // kOutBoth: O is still in tensor memory (the next item's first PV waits for epi_free)
       }
-      // This CTA's receive buffer is the V stage of the item's last tile (its
-      // last reader, that PV, has completed): arm the exchange barriers, then
-      // tell the partner that the buffer is ready.
-      float* recv = reinterpret_cast<float*>(sV + (glast & 1) * C::V_BYTES);
-      if (etid == 0) {
+      // Both V stages are free of this item's PV products: announce that this
+      // CTA's receive buffer is ready, with the exchange barrier armed first.
+      named_bar_sync(1, 128);
+      if (tid == 128) {
         mbar_arrive_expect_tx(&bars->exch_full, C::EXCH_BYTES);
-        mbar_arrive_expect_tx(&bars->ss_full, kBM * 4);
+        mbar_arrive_expect_tx(&bars->ss_full, kBM * 4);  // the partner's sums of squares, by st.async
         mbar_arrive_remote(map_to_cta(smem_u32(&bars->peer_ready), partner));
       }
-      const float inv = (rank == 0) ? 1.0f / lr.x : coef2 / lr.x;
-      // The half that goes to the partner: 32 columns at a time from tensor
-      // memory straight into its receive buffer (16-byte chunks of each row
-      // XOR-swizzled by the row, so that a warp's stores and loads spread over
-      // the banks).
-      const bool peer_ok = mbar_wait_acq_cluster(&bars->peer_ready, k & 1, wc);
-      const uint32_t dst_row = map_to_cta(smem_u32(recv + r * HALF), partner);
+      const float inv = (rank == 0) ? 1.0f / l_run : coef2 / l_run;
+      float* srow = stage + r * HALF;
 #pragma unroll
       for (int c = 0; c < HALF / 32; ++c) {
         uint32_t ov[32];
         tmem_ld32_sync(tl + C::TM_O + send0 + 32 * c, ov);
-        if (peer_ok) {
 #pragma unroll
-          for (int f = 0; f < 8; ++f) {
-            const int chunk = (c * 8 + f) ^ (r % NC);
-            st_async_v4(dst_row + chunk * 16, __uint_as_float(ov[4 * f + 0]) * inv,
-                        __uint_as_float(ov[4 * f + 1]) * inv, __uint_as_float(ov[4 * f + 2]) * inv,
-                        __uint_as_float(ov[4 * f + 3]) * inv, peer_exch);
-          }
+        for (int f = 0; f < 8; ++f) {
+          const int chunk = (c * 8 + f) ^ (r % NC);
+          *reinterpret_cast<float4*>(srow + chunk * 4) =
+              make_float4(__uint_as_float(ov[4 * f + 0]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                          __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
         }
       }
-      // the half this CTA keeps, in registers
+      fence_proxy_async_smem();  // the staged rows are read by the bulk copy (async proxy)
+      __syncwarp();
+      // the partner's receive buffer must be free before this CTA writes into it
+      const bool peer_ok = mbar_wait_acq_cluster(&bars->peer_ready, k & 1, wc);
+      if (lane == 0 && peer_ok) {
+        const int off = quarter * 32 * HALF;  // this warp's 32 rows, contiguous
+        bulk_copy_s2cluster(map_to_cta(smem_u32(recv + off), partner), stage + off, 32 * HALF * 4,
+                            map_to_cta(smem_u32(&bars->exch_full), partner));
+        bulk_commit_group();
+      }
+      mbar_wait(&bars->exch_full, k & 1, wdrain);  // the partner's half has landed (even after an abort)
       float y[HALF];
+      float ss = 0.f;
+      const float* rrow = recv + r * HALF;
 #pragma unroll
       for (int c = 0; c < HALF / 32; ++c) {
         uint32_t ov[32];
         tmem_ld32_sync(tl + C::TM_O + own0 + 32 * c, ov);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) y[32 * c + i] = __uint_as_float(ov[i]) * inv;
-      }
-      // O is drained: the next item's first PV may overwrite it
-      tc_fence_before();
-      named_bar_sync(2, 128);
-      if (etid == 0) mbar_arrive(&bars->o_free);
-      // the partner's half has landed (waited for even after an abort: the
-      // buffer was armed and announced above)
-      mbar_wait_acq_cluster(&bars->exch_full, k & 1, wdrain);
-      float ss = 0.f;
-      const float* rrow = recv + r * HALF;
+        for (int f = 0; f < 8; ++f) {
+          const int chunk = (c * 8 + f) ^ (r % NC);
+          const float4 xr = *reinterpret_cast<const float4*>(rrow + chunk * 4);
+          const float xs[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
-      for (int c4 = 0; c4 < NC; ++c4) {
-        const int chunk = c4 ^ (r % NC);
-        const float4 xr = *reinterpret_cast<const float4*>(rrow + chunk * 4);
-        y[4 * c4 + 0] += xr.x;
-        y[4 * c4 + 1] += xr.y;
-        y[4 * c4 + 2] += xr.z;
-        y[4 * c4 + 3] += xr.w;
-        ss = fmaf(y[4 * c4 + 0], y[4 * c4 + 0], ss);
-        ss = fmaf(y[4 * c4 + 1], y[4 * c4 + 1], ss);
-        ss = fmaf(y[4 * c4 + 2], y[4 * c4 + 2], ss);
-        ss = fmaf(y[4 * c4 + 3], y[4 * c4 + 3], ss);
+          for (int e = 0; e < 4; ++e) {
+            const float val = fmaf(__uint_as_float(ov[4 * f + e]), inv, xs[e]);
+            y[32 * c + 4 * f + e] = val;
+            ss = fmaf(val, val, ss);
+          }
+        }
       }
-      // the receive buffer is free again: the V producer may reload the stage
-      named_bar_sync(2, 128);
-      if (etid == 0) mbar_arrive(&bars->epi_free[k & 1]);
-      // this row's half of the sum of squares to the partner
-      if (peer_ok) st_async_f32(peer_ssx, ss, peer_ss);
+      // this row's half of the sum of squares to the partner: an asynchronous
+      // store that completes on the partner's barrier (armed before its
+      // receive buffer was announced)
+      if (peer_ok)
+        st_async_f32(map_to_cta(smem_u32(ssx + r), partner), ss, map_to_cta(smem_u32(&bars->ss_full), partner));
+      if (lane == 0 && peer_ok) bulk_wait_group_read0();  // the outgoing copy has left the staging rows
+      __syncwarp();
+      named_bar_sync(1, 128);  // every warp's outgoing copy is done with the rows the output tile reuses
       mbar_wait_acq_cluster(&bars->ss_full, k & 1, wdrain);
       const float rs = rsqrtf((ss + ssx[r]) / static_cast<float>(C::DV) + p.eps);
       const float gsc = (1.0f - p.lambda_init) * rs;
-      if (!peer_ok) ok = false;
-      // bf16 output, this CTA's columns of the row, straight to global memory (rows >= N skipped)
-      if (qrow < N && DA_CHECK(p.status, it.b >= 0 && it.b < p.B && it.h >= 0 && it.h < p.H)) {
-        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(it.b) * N + qrow) * p.H + it.h) * C::DV + own0;
+      // bf16 tile [64-column block][128 rows][64 columns], 128-byte swizzle, in the staging stage
+      const uint32_t sout = smem_u32(stage);
 #pragma unroll
-        for (int c8 = 0; c8 < HALF / 8; ++c8) {
-          uint32_t w4[4];
+      for (int c8 = 0; c8 < HALF / 8; ++c8) {
+        uint32_t w4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 8 * c8 + 2 * e;
-            w4[e] = pack_bf16x2(y[c] * gsc * __ldg(p.rms_w + own0 + c), y[c + 1] * gsc * __ldg(p.rms_w + own0 + c + 1));
-          }
-          st_global_v4(orow + 8 * c8, w4[0], w4[1], w4[2], w4[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int c = 8 * c8 + 2 * e;
+          w4[e] = pack_bf16x2(y[c] * gsc * __ldg(p.rms_w + own0 + c), y[c + 1] * gsc * __ldg(p.rms_w + own0 + c + 1));
         }
+        const uint32_t a = sout + (c8 / 8) * C::BLK_BYTES + r * 128 + (((c8 % 8) ^ (r & 7)) << 4);
+        st_shared_v4(a, w4[0], w4[1], w4[2], w4[3]);
       }
+      fence_proxy_async_smem();  // the tile is read by the TMA store (async proxy)
+      // hand the staged tile to warp 3, which stores it and frees the V stages,
+      // and go on with the next item
+      named_bar_arrive(2, 160);
     }
   }
 
@@ -727,24 +682,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int QKF, int OUT = kOutNorm>
 static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const PrefillParams& prm, cudaStream_t stream) {
+                            const CUtensorMap& to, const PrefillParams& prm, cudaStream_t stream, int ctl_dev = -1,
+                            unsigned long long ctl_ctx = 0) {
   using C = Cfg<D, QKF != kQkBf16>;
-  // per device and context: the shared-memory attribute is set and the
-  // resident cluster count looked up on the first launch only (again after a
-  // cudaDeviceReset, which creates a new context)
+  // per device and context: the shared-memory size and the cluster shape (a
+  // pair along x) are set as function attributes and the resident cluster
+  // count looked up on the first launch only (again after a cudaDeviceReset,
+  // which creates a new context).  A launch that carries no attributes costs
+  // the host about 0.6 us less than one that passes the cluster shape.
   static int max_clusters[64] = {};
   static unsigned long long set_ctx[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
+  int dev = ctl_dev;
+  cudaError_t e = cudaSuccess;
+  if (dev < 0 && (e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const unsigned long long ctx = current_context_id();
+  const unsigned long long ctx = ctl_ctx != 0 ? ctl_ctx : current_context_id();
   int& mc = max_clusters[dev];
   if (ctx == 0 || set_ctx[dev] != ctx) mc = 0;
   if (mc == 0) {
-    e = cudaFuncSetAttribute(prefill_sm100_kernel<D, QKF, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
+    const auto fn = prefill_sm100_kernel<D, QKF, OUT>;
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeRequiredClusterWidth, 2)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeRequiredClusterHeight, 1)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeRequiredClusterDepth, 1)) != cudaSuccess)
+      return e;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -767,10 +728,13 @@ static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
   }
   const int clusters = prm.n_items < mc ? prm.n_items : mc;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QKF, OUT>, tq, tk, tv, prm);
+  cfg.attrs = nullptr;  // the required cluster shape is the function's own
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<D, QKF, OUT>, tq, tk, tv, to, prm);
 }
 
-cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const CUtensorMap& to, void* o,
                                  int B, int N, int H, int d, int causal, const float* lambda, float lambda_init,
                                  const float* rms_w, float eps, int mode, const float* q_scale,
                                  const float* k_scale, int qk_bits, DevCtl ctl, cudaStream_t stream) {
@@ -798,17 +762,17 @@ cudaError_t launch_prefill_sm100(const CUtensorMap& tq, const CUtensorMap& tk, c
   prm.limit_ns = ctl.limit_ns;
   if (q_scale != nullptr) {
     if (d != 128) return cudaErrorInvalidValue;
-    if (qk_bits == 8) return launch_d<128, kQkE4m3>(tq, tk, tv, prm, stream);
-    if (qk_bits == 4) return launch_d<128, kQkE2m1>(tq, tk, tv, prm, stream);
+    if (qk_bits == 8) return launch_d<128, kQkE4m3>(tq, tk, tv, to, prm, stream, ctl.dev, ctl.ctx);
+    if (qk_bits == 4) return launch_d<128, kQkE2m1>(tq, tk, tv, to, prm, stream, ctl.dev, ctl.ctx);
     return cudaErrorInvalidValue;
   }
-  if (d == 128) return launch_d<128, kQkBf16>(tq, tk, tv, prm, stream);
-  if (d == 64) return launch_d<64, kQkBf16>(tq, tk, tv, prm, stream);
+  if (d == 128) return launch_d<128, kQkBf16>(tq, tk, tv, to, prm, stream, ctl.dev, ctl.ctx);
+  if (d == 64) return launch_d<64, kQkBf16>(tq, tk, tv, to, prm, stream, ctl.dev, ctl.ctx);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                       void* o, int B, int N, int H, int d, int causal,
+                                       const CUtensorMap* to, void* o, int B, int N, int H, int d, int causal,
                                        const float* lambda, float lambda_init, const float* rms_w, float eps, int mode,
                                        float* o_maps, float* lse, int n_pad, DevCtl ctl, cudaStream_t stream) {
   PrefillParams prm = {};
@@ -834,14 +798,14 @@ cudaError_t launch_prefill_sm100_stats(const CUtensorMap& tq, const CUtensorMap&
   prm.o_maps = o_maps;
   prm.lse = lse;
   prm.n_pad = n_pad;
-  if (o) {  // the normalised output as well
-    if (d == 128) return launch_d<128, kQkBf16, kOutBoth>(tq, tk, tv, prm, stream);
-    if (d == 64) return launch_d<64, kQkBf16, kOutBoth>(tq, tk, tv, prm, stream);
+  if (to) {  // the normalised output as well
+    if (d == 128) return launch_d<128, kQkBf16, kOutBoth>(tq, tk, tv, *to, prm, stream, ctl.dev, ctl.ctx);
+    if (d == 64) return launch_d<64, kQkBf16, kOutBoth>(tq, tk, tv, *to, prm, stream, ctl.dev, ctl.ctx);
     return cudaErrorInvalidValue;
   }
-  // statistics only
-  if (d == 128) return launch_d<128, kQkBf16, kOutStats>(tq, tk, tv, prm, stream);
-  if (d == 64) return launch_d<64, kQkBf16, kOutStats>(tq, tk, tv, prm, stream);
+  // statistics only: the output map is never used, tv stands in for it
+  if (d == 128) return launch_d<128, kQkBf16, kOutStats>(tq, tk, tv, tv, prm, stream, ctl.dev, ctl.ctx);
+  if (d == 64) return launch_d<64, kQkBf16, kOutStats>(tq, tk, tv, tv, prm, stream, ctl.dev, ctl.ctx);
   return cudaErrorInvalidValue;
 }
 

@@ -318,13 +318,34 @@ __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __rest
   const int first = chunk_start[s];
   int nch = chunk_start[s + 1] - first;
   if (!DA_CHECK(dbg, nch >= 1 && first >= 0 && first + nch <= chunk_start[gridDim.y])) nch = 0;
+  // The maxima over the chunks: each thread takes every 256th chunk, then a
+  // reduction over the block (one round of loads instead of one per chunk).
+  __shared__ float mx[2][kDV / 32];
   float M1 = -INFINITY, M2 = -INFINITY;
-  for (int i = 0; i < nch; ++i) {
+  for (int i = c; i < nch; i += kDV) {
     const float* r = ws + (static_cast<size_t>(first + i) * H + h) * kRecFloats;
     M1 = fmaxf(M1, r[0]);
     M2 = fmaxf(M2, r[2]);
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    M1 = fmaxf(M1, __shfl_xor_sync(0xffffffffu, M1, off));
+    M2 = fmaxf(M2, __shfl_xor_sync(0xffffffffu, M2, off));
+  }
+  if ((c & 31) == 0) {
+    mx[0][c >> 5] = M1;
+    mx[1][c >> 5] = M2;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kDV / 32; ++w) {
+    M1 = fmaxf(M1, mx[0][w]);
+    M2 = fmaxf(M2, mx[1][w]);
+  }
+  // The weighted sums: the chunks' loads do not depend on the sums, so the
+  // unrolled loop keeps several chunks' records in flight.
   float L1 = 0.f, L2 = 0.f, O1 = 0.f, O2 = 0.f;
+#pragma unroll 8
   for (int i = 0; i < nch; ++i) {
     const float* r = ws + (static_cast<size_t>(first + i) * H + h) * kRecFloats;
     const float f1 = fast_exp2(r[0] - M1), f2 = fast_exp2(r[2] - M2);

@@ -267,6 +267,36 @@ def test_full_size_64k_needle_sampled():
     assert torch.isfinite(y.float()).all()
 
 
+def _oracle_full_head(inp, b, h, block=1024):
+    """Every output row of one (batch, head), computed by the oracle in
+    blocks of query rows (the rows are independent: each block still scores
+    its queries against every key)."""
+    f = wl.to_f64
+    N = inp.q.shape[1]
+    lam = oracle_lambda(inp)
+    qh, kh, vh = (f(t[b:b + 1, :, h:h + 1]) for t in (inp.q, inp.k, inp.v))
+    w = f(inp.rms_w)
+    parts = [ref.diffattn_fwd(qh, kh, vh, lam, inp.lambda_init, w, inp.eps, inp.causal,
+                              rows=np.arange(r0, min(N, r0 + block)))[0, :, 0]
+             for r0 in range(0, N, block)]
+    return np.concatenate(parts, axis=0)
+
+
+@pytest.mark.parametrize("case,head", [("prefill_64k_needle", (0, 0)), ("prefill_13b_causal", (1, 19)),
+                                       ("prefill_13b_nomask", (0, 7))])
+def test_full_size_one_head_complete(case, head):
+    # one whole head of each long configuration, element by element: all N
+    # query rows against all keys (the 64K case takes the head whose needle
+    # key the last query aligns with)
+    inp = wl.make_prefill_case(case, device="cuda")
+    y, _ = run_prefill(inp)
+    b, h = head
+    got = wl.to_f64(y[b, :, h])
+    del y
+    torch.cuda.empty_cache()
+    assert_close(got, _oracle_full_head(inp, b, h))
+
+
 # ------------------------------------------------------------------ decode --
 
 def run_decode(inp, mode=api.MODE_DIFF):

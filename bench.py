@@ -620,6 +620,24 @@ def bench_small_prefill(api, wl, dev, reduce_max, barrier, rank, K=400):
     b.record()
     torch.cuda.synchronize()
     dev_ms = reduce_max(a.elapsed_time(b)) / K
+    # The same calls captured once in a CUDA graph (G launches) and replayed:
+    # a latency-bound loop then costs the host one graph launch per G calls.
+    G, reps = 100, 20
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cap = args[:-1] + (torch.cuda.current_stream().cuda_stream,)
+        assert all(L.diffattn_fwd(*cap) == api.OK for _ in range(G))
+    g.replay()
+    torch.cuda.synchronize()
+    t = time.perf_counter()
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    graph_host_us = (time.perf_counter() - t) / (reps * G) * 1e6
+    torch.cuda.synchronize()
+    graph_dev_ms = reduce_max(a.elapsed_time(b)) / (reps * G)
+    del g
     flops_alg = prefill_flops(B, N, H, d, True, "algorithmic")
     host = statistics.median(host_us)
     floor = statistics.median(floor_us)
@@ -627,11 +645,15 @@ def bench_small_prefill(api, wl, dev, reduce_max, barrier, rank, K=400):
             "host_us_per_call": host, "host_us_per_call_all": host_us,
             "ctypes_and_checks_us": floor, "library_launch_us": host - floor,
             "device_ms_per_launch": dev_ms, "achieved_tflops_algorithmic": flops_alg / (dev_ms * 1e-3) / 1e12,
+            "cuda_graph": {"launches_per_graph": G, "replays": reps, "host_us_per_launch": graph_host_us,
+                           "device_ms_per_launch": graph_dev_ms,
+                           "achieved_tflops_algorithmic": flops_alg / (graph_dev_ms * 1e-3) / 1e12},
             "how": "host: wall time of back-to-back diffattn_fwd calls through ctypes, no synchronisation inside; "
                    "ctypes_and_checks_us: the same with N = 0 (validation only, no tensor map, no launch); "
                    "library_launch_us: the difference (tensor-map lookup, launch); "
-                   "device: CUDA events around K back-to-back launches",
-            "gpu_launches": K + 20 + K}
+                   "device: CUDA events around K back-to-back launches; cuda_graph: the same call captured "
+                   "G times in one CUDA graph, replayed, host wall time and CUDA events per launch",
+            "gpu_launches": K + 20 + K + G * (reps + 1)}
 
 
 def run_reference(args):

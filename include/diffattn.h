@@ -32,6 +32,12 @@
  *    errors only; nothing is synchronised.  A kernel-side failure (a bounded
  *    wait that ran out) is recorded in a device status word that
  *    diffattn_device_status() reads.
+ *  - Calls may be captured in a CUDA graph (stream capture) and replayed:
+ *    each one enqueues only kernel launches and memsets on `stream`.  The
+ *    first call of an entry point on a device and context sets kernel
+ *    attributes and looks up occupancy, so make it once before capturing.
+ *    A replay reads the buffers the captured call was given, at their
+ *    current contents.
  *  - Tensors are dense and row-major in the layouts given below; every
  *    tensor pointer must be 16-byte aligned.
  *  - Return values are diffattn_status codes; 0 is success.

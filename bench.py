@@ -947,8 +947,24 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world
     alg = kv_bytes + io_bytes
     gbs = alg / (ms * 1e-3) / 1e9
     traffic = read_profile_traffic("decode_decode_64x12", alg)
+    # the same step captured in a CUDA graph and replayed (no host launch
+    # between the planning, partial and combine kernels)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    g.replay()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    g_ms = reduce_max(a.elapsed_time(b)) / steps
+    del g
     return {
         "metric": "decode HBM GB/s", "value": job_throughput(alg, world, ms) / 1e9, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+        "cuda_graph": {"ms_per_step": g_ms, "gbs": alg / (g_ms * 1e-3) / 1e9,
+                       "frac": alg / (g_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "workload": f"{name}: S={S} H={H} d={d} sum(L)={T} bf16 KV cache "
                     f"({kv_bytes / 1e9:.2f} GB per step)",
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -956,7 +972,7 @@ def bench_decode(api, wl, dev, peaks, peak_src, rank, reduce_max, barrier, world
                      "kernel": "decode_plan_kernel + decode_partial_kernel + decode_combine_kernel",
                      "algorithmic_bytes": alg, "peak_source": f"{peak_src} HBM copy"},
         "clocks": clk, "loop_wall_s": wall,
-        "gpu_launches": 3 * steps,  # planning, partial and combine kernels
+        "gpu_launches": 3 * steps + 3 * (steps + 1),  # planning, partial and combine kernels; eager, then graph
     }
 
 

@@ -24,7 +24,9 @@
 //     own online softmax state in the log2 domain.  The 4 warps merge, and
 //     the CTA writes (m1, l1, m2, l2, o1[256], o2[256]) for its chunk.
 //   * decode_combine_kernel: one CTA per (head, sequence) merges the
-//     sequence's chunks with the log-sum-exp rescale per map, forms
+//     sequence's chunks with the log-sum-exp rescale per map (four groups of
+//     256 threads, one thread per channel, each group a quarter of the
+//     chunks, then the groups' sums in a fixed order), forms
 //     o1/l1 - lambda o2/l2, and applies the RMSNorm and scale.
 // Workspace: the chunk records (room for S * ceil(max_seqlen / 512) chunks
 // per head), then the S + 1 chunk offsets and the work counter.
@@ -43,6 +45,8 @@ constexpr int kGroup = 8;               // keys in flight per warp
 constexpr int kKeysPerWarp = 128;
 constexpr int kChunk = kWarps * kKeysPerWarp;  // keys per CTA
 constexpr int kRecFloats = 4 + 2 * kDV;        // m1, l1, m2, l2, o1[256], o2[256]
+constexpr int kCombGroups = 4;                  // chunk groups the combine merges side by side
+constexpr int kCombThreads = kCombGroups * kDV;  // combine CTA: one thread per (group, channel)
 constexpr float kLog2e = 1.4426950408889634f;
 }  // namespace
 
@@ -307,22 +311,26 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
   }
 }
 
-__global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __restrict__ ws,
-                                                             const int* __restrict__ chunk_start, int H,
-                                                             __nv_bfloat16* __restrict__ o,
-                                                             const float* __restrict__ lambda_ptr, int mode,
-                                                             float lambda_init, const float* __restrict__ rms_w,
-                                                             float eps, int* dbg) {
+__global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const float* __restrict__ ws,
+                                                                      const int* __restrict__ chunk_start, int H,
+                                                                      __nv_bfloat16* __restrict__ o,
+                                                                      const float* __restrict__ lambda_ptr, int mode,
+                                                                      float lambda_init,
+                                                                      const float* __restrict__ rms_w, float eps,
+                                                                      int* dbg) {
   const int h = blockIdx.x, s = blockIdx.y;
-  const int c = threadIdx.x;
+  const int tid = threadIdx.x;
+  const int c = tid % kDV;     // output channel
+  const int grp = tid / kDV;   // chunk group: chunks grp, grp + kCombGroups, ...
   const int first = chunk_start[s];
   int nch = chunk_start[s + 1] - first;
   if (!DA_CHECK(dbg, nch >= 1 && first >= 0 && first + nch <= chunk_start[gridDim.y])) nch = 0;
-  // The maxima over the chunks: each thread takes every 256th chunk, then a
-  // reduction over the block (one round of loads instead of one per chunk).
-  __shared__ float mx[2][kDV / 32];
+  // The maxima over the chunks: each thread takes every kCombThreads-th
+  // chunk, then a reduction over the block (one round of loads instead of
+  // one per chunk).
+  __shared__ float mx[2][kCombThreads / 32];
   float M1 = -INFINITY, M2 = -INFINITY;
-  for (int i = c; i < nch; i += kDV) {
+  for (int i = tid; i < nch; i += kCombThreads) {
     const float* r = ws + (static_cast<size_t>(first + i) * H + h) * kRecFloats;
     M1 = fmaxf(M1, r[0]);
     M2 = fmaxf(M2, r[2]);
@@ -332,21 +340,21 @@ __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __rest
     M1 = fmaxf(M1, __shfl_xor_sync(0xffffffffu, M1, off));
     M2 = fmaxf(M2, __shfl_xor_sync(0xffffffffu, M2, off));
   }
-  if ((c & 31) == 0) {
-    mx[0][c >> 5] = M1;
-    mx[1][c >> 5] = M2;
+  if ((tid & 31) == 0) {
+    mx[0][tid >> 5] = M1;
+    mx[1][tid >> 5] = M2;
   }
   __syncthreads();
 #pragma unroll
-  for (int w = 0; w < kDV / 32; ++w) {
+  for (int w = 0; w < kCombThreads / 32; ++w) {
     M1 = fmaxf(M1, mx[0][w]);
     M2 = fmaxf(M2, mx[1][w]);
   }
-  // The weighted sums: the chunks' loads do not depend on the sums, so the
-  // unrolled loop keeps several chunks' records in flight.
+  // Each group's weighted sums over its chunks (the groups run side by side,
+  // so a long sequence's chain of loads is kCombGroups times shorter).
   float L1 = 0.f, L2 = 0.f, O1 = 0.f, O2 = 0.f;
-#pragma unroll 8
-  for (int i = 0; i < nch; ++i) {
+#pragma unroll 4
+  for (int i = grp; i < nch; i += kCombGroups) {
     const float* r = ws + (static_cast<size_t>(first + i) * H + h) * kRecFloats;
     const float f1 = fast_exp2(r[0] - M1), f2 = fast_exp2(r[2] - M2);
     L1 = fmaf(f1, r[1], L1);
@@ -354,19 +362,42 @@ __global__ void __launch_bounds__(kDV) decode_combine_kernel(const float* __rest
     O1 = fmaf(f1, r[4 + c], O1);
     O2 = fmaf(f2, r[4 + kDV + c], O2);
   }
-  const float ov = O1 / L1 + map2_coefficient(mode, *lambda_ptr) * (O2 / L2);  // c = -lambda, 0 or +lambda
+  __shared__ float po[2][kCombGroups][kDV];
+  __shared__ float pl[2][kCombGroups];
+  po[0][grp][c] = O1;
+  po[1][grp][c] = O2;
+  if (c == 0) {
+    pl[0][grp] = L1;
+    pl[1][grp] = L2;
+  }
+  __syncthreads();
+  // the groups' sums in a fixed order, by the first 256 threads
+  float ov = 0.f;
+  if (grp == 0) {
+    float o1 = 0.f, o2 = 0.f, l1 = 0.f, l2 = 0.f;
+#pragma unroll
+    for (int g = 0; g < kCombGroups; ++g) {
+      o1 += po[0][g][c];
+      o2 += po[1][g][c];
+      l1 += pl[0][g];
+      l2 += pl[1][g];
+    }
+    ov = o1 / l1 + map2_coefficient(mode, *lambda_ptr) * (o2 / l2);  // c = -lambda, 0 or +lambda
+  }
   // sum of squares over the 256 channels
   __shared__ float red[kDV / 32];
   float ss = ov * ov;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if ((c & 31) == 0) red[c >> 5] = ss;
+  if (grp == 0 && (c & 31) == 0) red[c >> 5] = ss;
   __syncthreads();
-  float tot = 0.f;
+  if (grp == 0) {
+    float tot = 0.f;
 #pragma unroll
-  for (int i = 0; i < kDV / 32; ++i) tot += red[i];
-  const float rs = rsqrtf(tot / static_cast<float>(kDV) + eps);
-  o[(static_cast<size_t>(s) * H + h) * kDV + c] = __float2bfloat16_rn((1.0f - lambda_init) * rms_w[c] * ov * rs);
+    for (int i = 0; i < kDV / 32; ++i) tot += red[i];
+    const float rs = rsqrtf(tot / static_cast<float>(kDV) + eps);
+    o[(static_cast<size_t>(s) * H + h) * kDV + c] = __float2bfloat16_rn((1.0f - lambda_init) * rms_w[c] * ov * rs);
+  }
 }
 
 namespace {
@@ -418,7 +449,7 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
       static_cast<const __nv_bfloat16*>(v_cache), cu_seqlens, S, max_seqlen, H, chunk_start, recs, dbg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<dim3(H, S), kDV, 0, stream>>>(recs, chunk_start, H, static_cast<__nv_bfloat16*>(o), lambda,
+  decode_combine_kernel<<<dim3(H, S), kCombThreads, 0, stream>>>(recs, chunk_start, H, static_cast<__nv_bfloat16*>(o), lambda,
                                                         mode, lambda_init, rms_w, eps, dbg);
   return cudaGetLastError();
 }

@@ -6,6 +6,8 @@ device status word.  Checked through the C ABI:
   * the parity cases of the release library (prefill bf16 and fp32, decode,
     low-bit queries and keys, the projections, the tensor-core backward) give
     the same results against the float64 oracle, and the status stays OK;
+  * the full-size prefill configurations and the decode workload pass every
+    check (status OK) and give the release library's results bit for bit;
   * a decode whose cu_seqlens gives a sequence more keys than max_seqlen (a
     host-built input that stays inside the cache: the kernels only ever read
     the first max_seqlen keys of a sequence) sets DIFFATTN_ERR_BOUNDS in the
@@ -130,6 +132,48 @@ def test_backward_under_debug_build():
         for x, w in zip(got[:3], want[:3]):
             assert np.linalg.norm(f(x) - w) / np.linalg.norm(w) <= 1e-2
     assert api.device_status() == api.OK
+
+
+def _release(fn):
+    """fn() run on the release library (the debug one is restored after)."""
+    _lib.use_debug_library(False)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+        assert api.device_status() == api.OK
+        return out
+    finally:
+        _lib.use_debug_library(True)
+
+
+@pytest.mark.parametrize("case", ["prefill_3b", "prefill_64k_needle", "prefill_13b_causal", "prefill_13b_nomask"])
+def test_full_size_prefill_under_debug_build(case):
+    # every tile, tail and grid position of the full-size launches passes the
+    # debug build's bounds checks, and the checks change no result
+    inp = wl.make_prefill_case(case, device="cuda")
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+
+    def run():
+        return api.diffattn_fwd(inp.q, inp.k, inp.v, lam, inp.lambda_init, inp.rms_w, inp.eps, inp.causal)
+
+    y = run()
+    torch.cuda.synchronize()
+    assert api.device_status() == api.OK
+    assert torch.equal(y, _release(run))
+
+
+def test_full_size_decode_under_debug_build():
+    inp = wl.make_decode_case("decode_64x12", device="cuda")
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+
+    def run():
+        return api.diffattn_decode(inp.q, inp.k_cache, inp.v_cache, inp.cu_seqlens, inp.max_seqlen, lam,
+                                   inp.lambda_init, inp.rms_w, inp.eps)
+
+    y = run()
+    torch.cuda.synchronize()
+    assert api.device_status() == api.OK
+    assert torch.equal(y, _release(run))
 
 
 def _overlong_decode():

@@ -6,8 +6,10 @@ device status word.  Checked through the C ABI:
   * the parity cases of the release library (prefill bf16 and fp32, decode,
     low-bit queries and keys, the projections, the tensor-core backward) give
     the same results against the float64 oracle, and the status stays OK;
-  * the full-size prefill configurations and the decode workload pass every
-    check (status OK) and give the release library's results bit for bit;
+  * the full-size prefill configurations, the decode workload, and the
+    backward and projections at the 3B-like shapes pass every check (status
+    OK) and give the release library's results (bit for bit where each
+    output element is written once);
   * a decode whose cu_seqlens gives a sequence more keys than max_seqlen (a
     host-built input that stays inside the cache: the kernels only ever read
     the first max_seqlen keys of a sequence) sets DIFFATTN_ERR_BOUNDS in the
@@ -174,6 +176,42 @@ def test_full_size_decode_under_debug_build():
     torch.cuda.synchronize()
     assert api.device_status() == api.OK
     assert torch.equal(y, _release(run))
+
+
+def test_full_size_backward_and_projections_under_debug_build():
+    # the tensor-core backward and both projection GEMMs at the 3B-like shapes:
+    # the checks pass and change nothing (dq, dk, dv and the projections are
+    # each written once, so bit for bit; dlambda and the norm weight's gradient
+    # are sums of per-CTA atomics, whose order varies)
+    inp = wl.make_prefill_case("prefill_3b", device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(3)
+    dy = torch.randn(inp.v.shape, generator=g, device="cuda").to(torch.bfloat16)
+    lam = api.diffattn_lambda(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.lambda_init)
+
+    def bwd():
+        return api.diffattn_bwd_tc(inp.q, inp.k, inp.v, dy, lam, inp.lambda_init, inp.rms_w, inp.eps, True)
+
+    got = bwd()
+    torch.cuda.synchronize()
+    assert api.device_status() == api.OK
+    want = _release(bwd)
+    for x, w in zip(got[:3], want[:3]):
+        assert torch.equal(x, w)
+    for x, w in zip(got[3:], want[3:]):
+        assert torch.allclose(x, w, rtol=1e-4, atol=1e-6)
+    del got, want, inp, dy
+    pj = wl.make_proj_case("proj_3b", device="cuda")
+    table = api.rope_table(pj.N, pj.d)
+
+    def proj():
+        q, k, v = api.qkv_proj(pj.x, pj.w_qkv, pj.B, pj.N, pj.H, pj.d, table)
+        return q, k, v, api.out_proj(v, pj.w_o)
+
+    got = proj()
+    torch.cuda.synchronize()
+    assert api.device_status() == api.OK
+    for x, w in zip(got, _release(proj)):
+        assert torch.equal(x, w)
 
 
 def _overlong_decode():

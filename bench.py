@@ -258,8 +258,11 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_rows_sample(inp, n_rows, seed=0):
-    """Run the float64 oracle on n_rows query rows of one head; returns seconds."""
+def oracle_rows_sample(inp, n_rows, seed=0, keep=None):
+    """Run the float64 oracle on n_rows query rows of one head; returns seconds.
+
+    With `keep` (a list), the sample (batch, head, rows, oracle output) is
+    appended to it."""
     import numpy as np
 
     import oracle.diffattn_ref as ref
@@ -273,29 +276,51 @@ def oracle_rows_sample(inp, n_rows, seed=0):
     qh, kh, vh = f(inp.q[b:b + 1, :, h:h + 1]), f(inp.k[b:b + 1, :, h:h + 1]), f(inp.v[b:b + 1, :, h:h + 1])
     lam = ref.lambda_reparam(f(inp.lq1), f(inp.lk1), f(inp.lq2), f(inp.lk2), inp.lambda_init)
     t0 = time.perf_counter()
-    ref.diffattn_fwd(qh, kh, vh, lam, inp.lambda_init, f(inp.rms_w), inp.eps, inp.causal, rows=rows)
-    return time.perf_counter() - t0
+    out = ref.diffattn_fwd(qh, kh, vh, lam, inp.lambda_init, f(inp.rms_w), inp.eps, inp.causal, rows=rows)
+    secs = time.perf_counter() - t0
+    if keep is not None:
+        keep.append((b, h, rows, out[0, :, 0]))
+    return secs
 
 
-def cpu_baseline(inp, budget_s):
-    """The oracle as it stands on a bounded sample of the workload (query rows of one head)."""
+def cpu_baseline(inp, budget_s, gpu_out=None):
+    """The oracle as it stands on a bounded sample of the workload (query rows of one head).
+
+    With `gpu_out` (the library's output for the same inputs), the sampled
+    rows double as a parity check: their errors against the oracle are
+    reported beside the bound the tests hold them to."""
+    import numpy as np
+
     N, d = inp.q.shape[1], inp.q.shape[4]
     rows = 256
-    t = oracle_rows_sample(inp, rows, seed=0)
+    keep = [] if gpu_out is not None else None
+    t = oracle_rows_sample(inp, rows, seed=0, keep=keep)
     rows_total, secs = rows, t
     seed = 1
     while secs < budget_s:
         n = int(min(N, max(64, rows * (budget_s - secs) / max(t, 1e-3) / 4)))
-        t = oracle_rows_sample(inp, n, seed=seed)
+        t = oracle_rows_sample(inp, n, seed=seed, keep=keep)
         rows_total += n
         secs += t
         seed += 1
     flops = rows_total * prefill_row_flops(N, d, inp.causal, "metric")
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-            "host_cpu_count": os.cpu_count(), "kind": "oracle",
-            "sample": f"{rows_total} query rows (each against all {N} keys, both maps materialised) of "
-                      f"{seed} seeded (batch, head) pairs of the {WORKLOAD} workload, {secs:.1f} s of CPU work; "
-                      f"FLOPs per row counted with the metric convention 16*N*d/2"}
+    res = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+           "host_cpu_count": os.cpu_count(), "kind": "oracle",
+           "sample": f"{rows_total} query rows (each against all {N} keys, both maps materialised) of "
+                     f"{seed} seeded (batch, head) pairs of the {WORKLOAD} workload, {secs:.1f} s of CPU work; "
+                     f"FLOPs per row counted with the metric convention 16*N*d/2"}
+    if keep:
+        num = den = mx = 0.0
+        for b, h, r, want in keep:
+            got = gpu_out[b, r, h].double().cpu().numpy()
+            num += float(((got - want) ** 2).sum())
+            den += float((want ** 2).sum())
+            mx = max(mx, float(np.abs(got - want).max()))
+        rel = (num / den) ** 0.5
+        res["parity"] = {"rows": rows_total, "rel_frobenius": rel, "max_abs": mx,
+                         "bound": {"rel_frobenius": 5e-3, "max_abs": 2e-2}, "pass": rel <= 5e-3 and mx <= 2e-2,
+                         "how": "the library's prefill on the same seeded inputs, against the oracle's rows above"}
+    return res
 
 
 # --------------------------------------------------------------- reference --
@@ -895,7 +920,13 @@ def run_ours(args):
     del inp, y
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_inp = wl.make_prefill_case(args.workload, seed=1234, device="cpu")
-        line["cpu_baseline"] = cpu_baseline(cpu_inp, args.cpu_budget_s)
+        # the library's output for the same tensors (one launch, outside every timed region)
+        g = {n: getattr(cpu_inp, n).to(dev) for n in ("q", "k", "v", "lq1", "lk1", "lq2", "lk2", "rms_w")}
+        g_lam = api.diffattn_lambda(g["lq1"], g["lk1"], g["lq2"], g["lk2"], cpu_inp.lambda_init)
+        g_out = api.diffattn_fwd(g["q"], g["k"], g["v"], g_lam, cpu_inp.lambda_init, g["rms_w"], cpu_inp.eps,
+                                 cpu_inp.causal).cpu()
+        del g, g_lam
+        line["cpu_baseline"] = cpu_baseline(cpu_inp, args.cpu_budget_s, g_out)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
